@@ -1,0 +1,229 @@
+"""ctypes front end of the CPU oracle (oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package entry point's smoke
+check and the benchmark's CPU-baseline leg import this module; the product
+path (dit_token_b200) never does.
+
+Every function takes numpy arrays of raw bf16 bit patterns (uint16) and
+returns new output arrays: the bf16 result (uint16, same layout as the input,
+padding rows left as given by ``out_init``) and, when asked for, the fp64
+result before rounding.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        # DIT_ORACLE_LIB lets the mutation tests load a deliberately broken copy.
+        path = os.environ.get("DIT_ORACLE_LIB") or _build.build()
+        L = ctypes.CDLL(path)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        L.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_f64.restype = f64
+        L.oracle_f64_to_bf16.argtypes = [f64]
+        L.oracle_f64_to_bf16.restype = ctypes.c_uint16
+        L.oracle_qk_rmsnorm_rope.argtypes = [
+            u16p, i64, u16p, i64, u16p, u16p, i32p, i32p, i32, i64, i32, i32, i32,
+            i32p, i32, i32, i32, f64, f64, u16p, u16p, f64p, f64p, i64p, i64]
+        L.oracle_adaln_modulate.argtypes = [
+            u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
+        L.oracle_gated_residual.argtypes = [
+            u16p, i64, u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
+        L.oracle_swiglu.argtypes = [
+            u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
+        for name in ("oracle_qk_rmsnorm_rope", "oracle_adaln_modulate",
+                     "oracle_gated_residual", "oracle_swiglu", "oracle_num_threads"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a, ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _u16(a):
+    a = np.asarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected raw bf16 bits as uint16, got {a.dtype}")
+    return a
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name}: invalid arguments (oracle returned {rc})")
+
+
+def _rows(rows):
+    if rows is None:
+        return None, 0
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    return r, r.size
+
+
+def _seqlens(cu_seqlens, cu_seqlens_padded):
+    cs = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    cp = np.ascontiguousarray(np.asarray(cu_seqlens_padded, dtype=np.int32))
+    return cs, cp
+
+
+def _flat_view(a, row_stride, rows_padded):
+    """The array as a flat uint16 buffer plus its row stride in elements."""
+    a = np.ascontiguousarray(_u16(a))
+    if row_stride is None:
+        row_stride = int(np.prod(a.shape[1:])) if a.ndim > 1 else 1
+    return a, row_stride
+
+
+def bf16_to_f64(bits: int) -> float:
+    return lib().oracle_bf16_to_f64(int(bits))
+
+
+def f64_to_bf16(x: float) -> int:
+    return int(lib().oracle_f64_to_bf16(float(x)))
+
+
+def f64_to_bf16_array(x) -> np.ndarray:
+    f = lib().oracle_f64_to_bf16
+    x = np.asarray(x, dtype=np.float64)
+    return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint16).reshape(x.shape)
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (bits << 16 is the binary32 value)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
+                    num_q_heads, num_k_heads, head_dim, rope_grid=None,
+                    sections=(0, 0, 0), rope_theta=10000.0, eps=1e-6,
+                    q_row_stride=None, k_row_stride=None, rows=None,
+                    q_out_init=None, k_out_init=None, want_f64=False):
+    """Per-head Q/K RMSNorm fused with 1D / 3D rotary embedding.
+
+    q, k: uint16 arrays whose first axis is the padded row; row strides
+    default to the product of the remaining axes.  Returns (q_out, k_out) or,
+    with want_f64, (q_out, k_out, q_f64, k_f64)."""
+    cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
+    B = cs.size - 1
+    q, qs = _flat_view(q, q_row_stride, None)
+    k, ks = _flat_view(k, k_row_stride, None)
+    nrows = q.shape[0]
+    q_out = np.array(q if q_out_init is None else q_out_init, dtype=np.uint16, copy=True)
+    k_out = np.array(k if k_out_init is None else k_out_init, dtype=np.uint16, copy=True)
+    q64 = np.full(q.shape, np.nan) if want_f64 else None
+    k64 = np.full(k.shape, np.nan) if want_f64 else None
+    grid = None if rope_grid is None else np.ascontiguousarray(np.asarray(rope_grid, dtype=np.int32))
+    wq = np.ascontiguousarray(_u16(q_weight))
+    wk = np.ascontiguousarray(_u16(k_weight))
+    r, nr = _rows(rows)
+    L = lib()
+    rc = L.oracle_qk_rmsnorm_rope(
+        _ptr(q, ctypes.c_uint16), qs, _ptr(k, ctypes.c_uint16), ks,
+        _ptr(wq, ctypes.c_uint16), _ptr(wk, ctypes.c_uint16),
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows,
+        num_q_heads, num_k_heads, head_dim,
+        _ptr(grid, ctypes.c_int32), *[int(s) for s in sections], float(rope_theta), float(eps),
+        _ptr(q_out, ctypes.c_uint16), _ptr(k_out, ctypes.c_uint16),
+        _ptr(q64, ctypes.c_double), _ptr(k64, ctypes.c_double),
+        _ptr(r, ctypes.c_int64), nr)
+    _check(rc, "qk_rmsnorm_rope")
+    if want_f64:
+        return q_out, k_out, q64, k64
+    return q_out, k_out
+
+
+def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
+                   mod_seq_stride=None, x_row_stride=None, rows=None, out_init=None,
+                   want_f64=False):
+    """out = LayerNorm(x) * (1 + scale_b) + shift_b on valid rows.
+
+    shift, scale: uint16 arrays [num_seqs, ...] read with mod_seq_stride
+    elements between sequences (default: hidden)."""
+    cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
+    B = cs.size - 1
+    x, xs = _flat_view(x, x_row_stride, None)
+    nrows = x.shape[0]
+    out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
+    o64 = np.full(out.shape, np.nan) if want_f64 else None
+    sh = np.ascontiguousarray(_u16(shift))
+    sc = np.ascontiguousarray(_u16(scale))
+    mss = hidden if mod_seq_stride is None else mod_seq_stride
+    r, nr = _rows(rows)
+    rc = lib().oracle_adaln_modulate(
+        _ptr(x, ctypes.c_uint16), xs, _ptr(sh, ctypes.c_uint16), _ptr(sc, ctypes.c_uint16), mss,
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
+        _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
+    _check(rc, "adaln_modulate")
+    return (out, o64) if want_f64 else out
+
+
+def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_seq_stride=None,
+                   x_row_stride=None, y_row_stride=None, rows=None, out_init=None,
+                   want_f64=False):
+    """out = x + gate_b * y on valid rows."""
+    cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
+    B = cs.size - 1
+    x, xs = _flat_view(x, x_row_stride, None)
+    y, ys = _flat_view(y, y_row_stride, None)
+    nrows = x.shape[0]
+    out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
+    o64 = np.full(out.shape, np.nan) if want_f64 else None
+    g = np.ascontiguousarray(_u16(gate))
+    gss = hidden if gate_seq_stride is None else gate_seq_stride
+    r, nr = _rows(rows)
+    rc = lib().oracle_gated_residual(
+        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _ptr(g, ctypes.c_uint16), gss,
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
+        _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
+    _check(rc, "gated_residual")
+    return (out, o64) if want_f64 else out
+
+
+def swiglu(a, b, cu_seqlens, cu_seqlens_padded, *, inner, a_row_stride=None, b_row_stride=None,
+           out_row_stride=None, nrows=None, rows=None, out_init=None, want_f64=False):
+    """out = silu(a) * b on valid rows.
+
+    a, b: uint16 arrays whose first axis is the padded row (for a chunked
+    [rows, 2*inner] buffer pass its two column halves).  The output has
+    ``out_row_stride`` (default ``inner``) elements per row; rows the oracle
+    does not write keep ``out_init`` (default: the bf16 NaN 0x7FC1)."""
+    cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
+    B = cs.size - 1
+    a, as_ = _flat_view(a, a_row_stride, None)
+    b, bs = _flat_view(b, b_row_stride, None)
+    n = a.shape[0] if nrows is None else nrows
+    ostride = inner if out_row_stride is None else out_row_stride
+    if out_init is None:
+        out = np.full((n, ostride), 0x7FC1, dtype=np.uint16)
+    else:
+        out = np.array(out_init, dtype=np.uint16, copy=True)
+    o64 = np.full(out.shape, np.nan) if want_f64 else None
+    r, nr = _rows(rows)
+    rc = lib().oracle_swiglu(
+        _ptr(a, ctypes.c_uint16), as_, _ptr(b, ctypes.c_uint16), bs,
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, n, inner,
+        _ptr(out, ctypes.c_uint16), ostride, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
+    _check(rc, "swiglu")
+    return (out, o64) if want_f64 else out

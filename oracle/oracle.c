@@ -1,0 +1,374 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for the fused per-token operators
+ * of a packed audio-video diffusion-transformer block.
+ *
+ * TEST INFRASTRUCTURE ONLY: used by the tests, the smoke check and the
+ * benchmark's CPU-baseline leg; never by the product path.  It shares no code
+ * with the CUDA library.  Each function below is the textbook definition of
+ * its operator written out with scalar loops, in the order the definition
+ * states it; the only parallelism is an OpenMP loop over independent rows.
+ *
+ * Pages: "Why Real-Time MiniMax H3 Serving Requires More Than a Faster DiT",
+ * "Key takeaways" bullets 1-2; "MiniMax H3 通过 vLLM-Omni 实现 FastH3 实时推理",
+ * "vLLM-Omni 中的系统级优化" bullets 1-2.  Those passages name the operators
+ * and the padding-free packed sequence but print no formula, so every formula
+ * here is the plainest standard reading (see the per-function comments).
+ *
+ * Parity pins: every function is pinned by the CPU tests (closed forms,
+ * invariants, library special cases); none is "parity unpinned".
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stddef.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ bf16 */
+
+double oracle_bf16_to_f64(uint16_t h)
+{
+    /* A bf16 value is the upper half of an IEEE binary32 value. */
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+uint16_t oracle_f64_to_bf16(double x)
+{
+    /* bf16: 1 sign bit, 8 exponent bits (bias 127), 7 stored mantissa bits.
+     * Between 2^e and 2^(e+1) (e >= -126) the spacing is 2^(e-7); below the
+     * smallest normal 2^-126 the spacing stays 2^-133 (subnormals).  Round
+     * |x| to the nearest multiple of that spacing with ties to even
+     * (nearbyint in the default rounding mode), then read off the bits of
+     * the now exactly representable value. */
+    if (isnan(x))
+        return signbit(x) ? 0xFFC0u : 0x7FC0u;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double ax = fabs(x);
+    if (isinf(ax))
+        return sign | 0x7F80u;
+    if (ax == 0.0)
+        return sign;
+    int e = ilogb(ax);
+    if (e < -126)
+        e = -126;
+    double spacing = ldexp(1.0, e - 7);
+    double r = nearbyint(ax / spacing) * spacing;
+    if (r >= ldexp(1.0, 128))
+        return sign | 0x7F80u; /* rounds past the largest finite bf16 */
+    float f = (float)r;        /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return sign | (uint16_t)(u >> 16);
+}
+
+static double ld(const uint16_t* p) { return oracle_bf16_to_f64(*p); }
+
+/* -------------------------------------------------------- packed rows */
+
+/* The padded buffer holds num_seqs sequences; sequence b owns padded rows
+ * [cu_seqlens_padded[b], cu_seqlens_padded[b+1]) and its first
+ * cu_seqlens[b+1] - cu_seqlens[b] rows are valid (the rest is structural
+ * suffix padding, which is neither read nor written).  Returns 1 and fills
+ * (*seq, *local) for a valid row, 0 for padding. */
+static int locate_row(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                      int32_t num_seqs, int64_t row, int32_t* seq, int64_t* local)
+{
+    for (int32_t b = 0; b < num_seqs; ++b) {
+        if (row >= cu_seqlens_padded[b] && row < cu_seqlens_padded[b + 1]) {
+            int64_t r = row - cu_seqlens_padded[b];
+            int64_t len = (int64_t)cu_seqlens[b + 1] - cu_seqlens[b];
+            if (r < len) {
+                *seq = b;
+                *local = r;
+                return 1;
+            }
+            return 0;
+        }
+    }
+    return 0;
+}
+
+static int64_t row_at(const int64_t* rows, int64_t i) { return rows ? rows[i] : i; }
+
+static int seqlens_ok(const int32_t* cs, const int32_t* cp, int32_t num_seqs, int64_t num_rows_padded)
+{
+    if (num_seqs < 0 || num_rows_padded < 0)
+        return 0;
+    if (num_seqs == 0)
+        return 1;
+    if (!cs || !cp || cs[0] != 0 || cp[0] != 0)
+        return 0;
+    for (int32_t b = 0; b < num_seqs; ++b) {
+        if (cs[b + 1] < cs[b] || cp[b + 1] < cp[b])
+            return 0;
+        if (cs[b + 1] - cs[b] > cp[b + 1] - cp[b])
+            return 0;
+    }
+    return cp[num_seqs] <= num_rows_padded;
+}
+
+static void put(uint16_t* out_bits, double* out_f64, int64_t idx, double v)
+{
+    out_bits[idx] = oracle_f64_to_bf16(v);
+    if (out_f64)
+        out_f64[idx] = v;
+}
+
+/* ------------------------------------------------------------ rotary */
+
+/* Rotation angle of pair j (elements 2j, 2j+1) of a head of width head_dim.
+ * 1D rows: angle = p * theta^(-2j/head_dim), the standard rotary frequency.
+ * 3D rows: head_dim is split into sections of sec_t, sec_h, sec_w elements
+ * (in that order); pair j lies in the section of axis s with width d_s and
+ * local pair index j', and rotates by p_s * theta^(-2j'/d_s). */
+static double rope_angle(int j, int head_dim, int is3d, const int64_t pos3[3], int64_t pos1,
+                         const int32_t sec[3], double theta)
+{
+    if (!is3d)
+        return (double)pos1 * pow(theta, -2.0 * (double)j / (double)head_dim);
+    int first = 0; /* first pair of the current section */
+    for (int s = 0; s < 3; ++s) {
+        int npairs = sec[s] / 2;
+        if (j < first + npairs) {
+            int jl = j - first;
+            return (double)pos3[s] * pow(theta, -2.0 * (double)jl / (double)sec[s]);
+        }
+        first += npairs;
+    }
+    return 0.0; /* unreachable when the sections sum to head_dim */
+}
+
+/* One head: RMSNorm over head_dim, times the weight, then rotate every
+ * interleaved pair (2j, 2j+1) by its angle:
+ *   ms    = (1/D) * sum_i x_i^2
+ *   y_i   = x_i / sqrt(ms + eps) * w_i
+ *   o_2j   = y_2j cos(a_j) - y_2j+1 sin(a_j)
+ *   o_2j+1 = y_2j sin(a_j) + y_2j+1 cos(a_j) */
+static void rmsnorm_rope_head(const uint16_t* x, const uint16_t* w, int D, double eps,
+                              int is3d, const int64_t pos3[3], int64_t pos1,
+                              const int32_t sec[3], double theta,
+                              uint16_t* out_bits, double* out_f64, double* y)
+{
+    double ms = 0.0;
+    for (int i = 0; i < D; ++i)
+        ms += ld(&x[i]) * ld(&x[i]);
+    ms /= (double)D;
+    double inv_rms = 1.0 / sqrt(ms + eps);
+    for (int i = 0; i < D; ++i)
+        y[i] = ld(&x[i]) * inv_rms * ld(&w[i]);
+    for (int j = 0; j < D / 2; ++j) {
+        double a = rope_angle(j, D, is3d, pos3, pos1, sec, theta);
+        double c = cos(a), s = sin(a);
+        double y0 = y[2 * j], y1 = y[2 * j + 1];
+        put(out_bits, out_f64, 2 * j, y0 * c - y1 * s);
+        put(out_bits, out_f64, 2 * j + 1, y0 * s + y1 * c);
+    }
+}
+
+int oracle_qk_rmsnorm_rope(
+    const uint16_t* q, int64_t q_row_stride,
+    const uint16_t* k, int64_t k_row_stride,
+    const uint16_t* q_weight, const uint16_t* k_weight,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded,
+    int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+    const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+    double rope_theta, double eps,
+    uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    if (!q || !k || !q_weight || !k_weight || !q_out || !k_out)
+        return -1;
+    if (head_dim <= 0 || head_dim % 2 || head_dim > 1024 || num_q_heads < 0 || num_k_heads < 0)
+        return -1;
+    if (q_row_stride < (int64_t)num_q_heads * head_dim || k_row_stride < (int64_t)num_k_heads * head_dim)
+        return -1;
+    const int32_t sec[3] = {sec_t, sec_h, sec_w};
+    if (rope_grid) {
+        for (int s = 0; s < 3; ++s)
+            if (sec[s] < 0 || sec[s] % 2)
+                return -1;
+        if (sec_t + sec_h + sec_w != head_dim)
+            return -1;
+    }
+    if (!seqlens_ok(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded))
+        return -1;
+    int64_t n = rows ? num_rows : num_rows_padded;
+
+#pragma omp parallel
+    {
+        double y[1024];
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t i = 0; i < n; ++i) {
+            int64_t row = row_at(rows, i), r;
+            int32_t b;
+            if (row < 0 || row >= num_rows_padded)
+                continue;
+            if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
+                continue;
+            /* Positions: a row inside the sequence's T x H x W video grid
+             * (t-major, then h, then w) takes 3D positions; every other row
+             * takes the 1D position counted from the end of the grid. */
+            int is3d = 0;
+            int64_t pos3[3] = {0, 0, 0}, pos1 = r;
+            if (rope_grid) {
+                int64_t T = rope_grid[3 * b], H = rope_grid[3 * b + 1], W = rope_grid[3 * b + 2];
+                int64_t thw = T * H * W;
+                if (r < thw) {
+                    is3d = 1;
+                    pos3[0] = r / (H * W);
+                    pos3[1] = (r / W) % H;
+                    pos3[2] = r % W;
+                } else {
+                    pos1 = r - thw;
+                }
+            }
+            for (int32_t h = 0; h < num_q_heads; ++h) {
+                int64_t off = row * q_row_stride + (int64_t)h * head_dim;
+                rmsnorm_rope_head(q + off, q_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta,
+                                  q_out + off, q_out_f64 ? q_out_f64 + off : NULL, y);
+            }
+            for (int32_t h = 0; h < num_k_heads; ++h) {
+                int64_t off = row * k_row_stride + (int64_t)h * head_dim;
+                rmsnorm_rope_head(k + off, k_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta,
+                                  k_out + off, k_out_f64 ? k_out_f64 + off : NULL, y);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------- adaLN */
+
+int oracle_adaln_modulate(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* shift, const uint16_t* scale, int64_t mod_seq_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    if (!x || !shift || !scale || !out || hidden <= 0)
+        return -1;
+    if (x_row_stride < hidden || out_row_stride < hidden || mod_seq_stride < 0)
+        return -1;
+    if (!seqlens_ok(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded))
+        return -1;
+    int64_t n = rows ? num_rows : num_rows_padded;
+
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t row = row_at(rows, i), r;
+        int32_t b;
+        if (row < 0 || row >= num_rows_padded)
+            continue;
+        if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
+            continue;
+        const uint16_t* xr = x + row * x_row_stride;
+        const uint16_t* sh = shift + (int64_t)b * mod_seq_stride;
+        const uint16_t* sc = scale + (int64_t)b * mod_seq_stride;
+        /* LayerNorm without affine: mean, then the biased variance about it. */
+        double mean = 0.0;
+        for (int32_t c = 0; c < hidden; ++c)
+            mean += ld(&xr[c]);
+        mean /= (double)hidden;
+        double var = 0.0;
+        for (int32_t c = 0; c < hidden; ++c)
+            var += (ld(&xr[c]) - mean) * (ld(&xr[c]) - mean);
+        var /= (double)hidden;
+        double inv_std = 1.0 / sqrt(var + eps);
+        /* Modulation: x_hat * (1 + scale) + shift. */
+        for (int32_t c = 0; c < hidden; ++c) {
+            double xhat = (ld(&xr[c]) - mean) * inv_std;
+            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);
+            put(out, out_f64, row * out_row_stride + c, v);
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------- gated residual */
+
+int oracle_gated_residual(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const uint16_t* gate, int64_t gate_seq_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    if (!x || !y || !gate || !out || hidden <= 0)
+        return -1;
+    if (x_row_stride < hidden || y_row_stride < hidden || out_row_stride < hidden || gate_seq_stride < 0)
+        return -1;
+    if (!seqlens_ok(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded))
+        return -1;
+    int64_t n = rows ? num_rows : num_rows_padded;
+
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t row = row_at(rows, i), r;
+        int32_t b;
+        if (row < 0 || row >= num_rows_padded)
+            continue;
+        if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
+            continue;
+        const uint16_t* g = gate + (int64_t)b * gate_seq_stride;
+        for (int32_t c = 0; c < hidden; ++c) {
+            double v = ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]);
+            put(out, out_f64, row * out_row_stride + c, v);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------- SwiGLU */
+
+int oracle_swiglu(
+    const uint16_t* a, int64_t a_row_stride,
+    const uint16_t* b, int64_t b_row_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t inner,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    if (!a || !b || !out || inner <= 0)
+        return -1;
+    if (a_row_stride < inner || b_row_stride < inner || out_row_stride < inner)
+        return -1;
+    if (!seqlens_ok(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded))
+        return -1;
+    int64_t n = rows ? num_rows : num_rows_padded;
+
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t row = row_at(rows, i), r;
+        int32_t s;
+        if (row < 0 || row >= num_rows_padded)
+            continue;
+        if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &s, &r))
+            continue;
+        for (int32_t c = 0; c < inner; ++c) {
+            double av = ld(&a[row * a_row_stride + c]);
+            double bv = ld(&b[row * b_row_stride + c]);
+            double silu = av / (1.0 + exp(-av));
+            put(out, out_f64, row * out_row_stride + c, silu * bv);
+        }
+    }
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

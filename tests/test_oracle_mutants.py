@@ -1,0 +1,76 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a private copy of oracle/oracle.c (a dropped
+term, a wrong sign or index, a transposed operand), builds it on the CPU, and
+runs the pin tests against it: every mutant must make at least one pin fail.
+"""
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
+        "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py"]
+
+# (name, original text, planted mistake)
+MUTANTS = [
+    ("rope_sign", "y0 * c - y1 * s", "y0 * c + y1 * s"),
+    ("rope_half_split_read", "double y0 = y[2 * j], y1 = y[2 * j + 1];",
+     "double y0 = y[j], y1 = y[j + D / 2];"),
+    ("rms_eps_dropped", "sqrt(ms + eps)", "sqrt(ms)"),
+    ("rms_mean_not_divided", "ms /= (double)D;", ""),
+    ("rms_weight_dropped", "y[i] = ld(&x[i]) * inv_rms * ld(&w[i]);", "y[i] = ld(&x[i]) * inv_rms;"),
+    ("rope_3d_freq_whole_head", "(double)jl / (double)sec[s]", "(double)jl / (double)head_dim"),
+    ("rope_3d_h_index", "pos3[1] = (r / W) % H;", "pos3[1] = (r / H) % W;"),
+    ("rope_tail_position", "pos1 = r - thw;", "pos1 = r;"),
+    ("rope_k_uses_q_weight", "rmsnorm_rope_head(k + off, k_weight,", "rmsnorm_rope_head(k + off, q_weight,"),
+    ("adaln_scale_without_one", "xhat * (1.0 + ld(&sc[c]))", "xhat * ld(&sc[c])"),
+    ("adaln_unbiased_variance", "var /= (double)hidden;", "var /= (double)(hidden - 1);"),
+    ("adaln_shift_scale_swapped", "double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);",
+     "double v = xhat * (1.0 + ld(&sh[c])) + ld(&sc[c]);"),
+    ("gate_dropped", "ld(&g[c]) * ld(&y[row * y_row_stride + c])", "ld(&y[row * y_row_stride + c])"),
+    ("gate_not_per_sequence", "gate + (int64_t)b * gate_seq_stride", "gate"),
+    ("silu_sign", "exp(-av)", "exp(av)"),
+    ("swiglu_operands_transposed", "double silu = av / (1.0 + exp(-av));\n            put(out, out_f64, row * out_row_stride + c, silu * bv);",
+     "double silu = bv / (1.0 + exp(-bv));\n            put(out, out_f64, row * out_row_stride + c, silu * av);"),
+    ("bf16_truncates", "nearbyint(ax / spacing)", "floor(ax / spacing)"),
+    ("padding_row_read", "if (r < len) {", "if (r <= len) {"),
+    ("rows_located_by_valid_offsets", "if (row >= cu_seqlens_padded[b] && row < cu_seqlens_padded[b + 1]) {",
+     "if (row >= cu_seqlens[b] && row < cu_seqlens[b + 1]) {"),
+]
+
+
+def _run_mutant(name, old, new, workdir):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"{name}: pattern not found in oracle.c"
+    d = os.path.join(workdir, name)
+    os.makedirs(d)
+    shutil.copy(os.path.join(ROOT, "oracle", "oracle.h"), d)
+    with open(os.path.join(d, "oracle.c"), "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(d, "liboracle.so")
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+                           "-o", lib, os.path.join(d, "oracle.c"), "-lm"])
+    env = dict(os.environ, DIT_ORACLE_LIB=lib, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *PINS],
+                       cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True,
+                       timeout=600)
+    return name, r.returncode, r.stdout[-400:]
+
+
+def test_every_planted_mistake_fails_a_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
+            results = list(ex.map(lambda m: _run_mutant(*m, tmp), MUTANTS))
+    survivors = [(n, out) for n, rc, out in results if rc == 0]
+    assert not survivors, f"mutants not caught by any pin: {survivors}"
+    # a clean copy must pass (the harness itself is sound)
+    with tempfile.TemporaryDirectory() as tmp:
+        name, rc, out = _run_mutant("clean", "int oracle_num_threads(void)", "int oracle_num_threads(void)", tmp)
+    assert rc == 0, out
