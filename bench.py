@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Throughput of the fused DiT token operators on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dit|reference]
+                    [--workload batched_varlen] [--seed 0]
+
+One step runs the whole per-token hot path once over one packed batch:
+Q/K RMSNorm + RoPE (in place), adaLN modulation, gated residual and SwiGLU,
+each on its own synthetic buffers of the workload's shapes.  The default
+workload is the largest single-GPU one, "batched_varlen": 4 requests with
+seeded lengths in [1024, 30000] (69,829 valid tokens at seed 0), hidden 5120,
+40 heads x 128, SwiGLU inner 13824, 3D RoPE on 24x42 latent frames plus a 1D
+tail.  Every op's working set (>= 1.4 GB) is larger than the 126 MB L2, so no
+flush is needed between steps.
+
+Timing: W untimed steps, then exactly K steps between CUDA events on the
+launch stream, a barrier + synchronize on both sides, the max over ranks.
+Rank 0 prints one JSON line.  ``value`` is tokens/s over all ranks; ``e2e``
+repeats the measurement through the same public API with the inputs copied
+from pinned host memory and the outputs copied back inside the timed region;
+``roofline`` rates the dominant kernel against the measured HBM copy
+bandwidth; ``cpu_baseline`` times the plain CPU oracle on a bounded sample.
+
+``--impl reference`` times the CPU oracle alone (the only reference this
+operator set has): rank 0 runs K + W bounded samples of the same workload on
+the host cores and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from dit_token_b200 import workloads as W  # noqa: E402
+
+METRIC = "fused DiT token-op throughput (tokens/s, achieved HBM GB/s, % of roofline) on 1 B200"
+UNIT = "tokens/s"
+OPS = ("qk_rmsnorm_rope", "adaln_modulate", "gated_residual", "swiglu")
+FALLBACK_HBM_GBS = 6650.0
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+# ------------------------------------------------------------ accounting
+
+def algorithmic_bytes(w: W.Workload) -> dict:
+    """HBM bytes each op must move per step: valid rows only, bf16.
+    qk: q and k read + written (4 bytes per element of each); adaLN: x read,
+    out written (4 C); gated residual: x, y read, out written (6 C); SwiGLU:
+    a, b read, out written (6 I).  Per-sequence vectors, norm weights and the
+    packing descriptors are O(num_seqs * C) and left out."""
+    n = w.num_valid
+    qk_elems = (w.num_q_heads + w.num_k_heads) * w.head_dim
+    return {"qk_rmsnorm_rope": 4 * qk_elems * n, "adaln_modulate": 4 * w.hidden * n,
+            "gated_residual": 6 * w.hidden * n, "swiglu": 6 * w.inner * n}
+
+
+def kernel_source_digest(op: str) -> str:
+    path = os.path.join(ROOT, "dit_token_b200", "csrc", f"{op}.cu")
+    h = hashlib.sha256()
+    for p in (path, os.path.join(ROOT, "dit_token_b200", "csrc", "common.cuh")):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(op: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel changed since."""
+    path = os.path.join(PROFILES, f"{op}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    d = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", text)
+    if not m or not d or d.group(1) != kernel_source_digest(op):
+        return None
+    return float(m.group(1))
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of one GPU while the work runs."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.samples = []
+        self.proc = None
+        try:
+            ident = str(torch.cuda.get_device_properties(device).uuid)
+            ident = ident if ident.startswith("GPU-") else "GPU-" + ident
+        except Exception:
+            ident = str(device)
+        self.ident = ident
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 f"--id={self.ident}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        window = [p for t, p in self.samples if t0 <= t <= t1 + 0.25]
+        rows = window or [p for _, p in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "in_timed_window": bool(window)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def data_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch (same lengths, different values)."""
+    return seed + 1000003 * rank
+
+
+def reduce_max(value: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------ GPU arm
+
+class Step:
+    """Device buffers of one step and the four calls through the binding."""
+
+    def __init__(self, w: W.Workload, host: dict, device):
+        import dit_token_b200 as dit
+        self.dit = dit
+        self.w = w
+        dev = lambda t: t.to(device, non_blocking=False)
+        self.cs = torch.from_numpy(w.cu_seqlens).to(device)
+        self.cp = torch.from_numpy(w.cu_seqlens_padded).to(device)
+        self.grid = None if w.rope_grid is None else torch.from_numpy(w.rope_grid).to(device)
+        self.q, self.k = dev(host["qk"]["q"]), dev(host["qk"]["k"])
+        self.wq, self.wk = dev(host["qk"]["q_weight"]), dev(host["qk"]["k_weight"])
+        self.ax, self.aout = dev(host["adaln"]["x"]), dev(host["adaln"]["out"])
+        self.mod = dev(host["adaln"]["mod"])
+        self.rx, self.ry, self.rout = dev(host["res"]["x"]), dev(host["res"]["y"]), dev(host["res"]["out"])
+        self.ab, self.sout = dev(host["swiglu"]["ab"]), dev(host["swiglu"]["out"])
+
+    def inputs(self):
+        """(device tensor, name) of every input the step consumes."""
+        return [(self.q, "q"), (self.k, "k"), (self.ax, "adaln_x"), (self.rx, "res_x"), (self.ry, "res_y"),
+                (self.ab, "ab")]
+
+    def outputs(self):
+        return [(self.q, "q"), (self.k, "k"), (self.aout, "adaln_out"), (self.rout, "res_out"),
+                (self.sout, "swiglu_out")]
+
+    def run(self, events=None):
+        w, d, rv = self.w, self.dit, W.rows_view
+        ev = events or {}
+        def mark(op, i):
+            if op in ev:
+                ev[op][i].record()
+        mark("qk_rmsnorm_rope", 0)
+        d.dit_qk_rmsnorm_rope(rv(self.q), rv(self.k), self.wq, self.wk, self.cs, self.cp,
+                              num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
+                              rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps)
+        mark("qk_rmsnorm_rope", 1)
+        mark("adaln_modulate", 0)
+        d.dit_adaln_modulate(rv(self.ax), self.mod[:, 0], self.mod[:, 1], self.cs, self.cp, out=rv(self.aout),
+                             eps=w.eps)
+        mark("adaln_modulate", 1)
+        mark("gated_residual", 0)
+        d.dit_gated_residual(rv(self.rx), rv(self.ry), self.mod[:, 2], self.cs, self.cp, out=rv(self.rout))
+        mark("gated_residual", 1)
+        mark("swiglu", 0)
+        ab = rv(self.ab)
+        d.dit_swiglu(ab[:, : w.inner], ab[:, w.inner:], self.cs, self.cp, out=rv(self.sout))
+        mark("swiglu", 1)
+
+
+def host_inputs(w: W.Workload) -> dict:
+    qk = W.qk_inputs(w)
+    adaln = W.adaln_inputs(w)
+    res = W.residual_inputs(w)
+    res["mod"] = adaln["mod"]
+    return {"qk": qk, "adaln": adaln, "res": res, "swiglu": W.swiglu_inputs(w)}
+
+
+def time_device(step: Step, steps: int, warmup: int, device):
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        step.run()
+    per_op = {op: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)] for op in OPS}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(device)
+    t_host0 = time.time()
+    start.record(stream)
+    for i in range(steps):
+        step.run({op: per_op[op][i] for op in OPS})
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    t_host1 = time.time()
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    op_ms = {op: statistics.fmean(a.elapsed_time(b) for a, b in per_op[op]) for op in OPS}
+    return elapsed_ms, op_ms, (t_host0, t_host1)
+
+
+def time_e2e(step: Step, steps: int, warmup: int, device):
+    """Same step through the public API, inputs copied from pinned host memory
+    and results copied back to pinned host memory inside the timed region."""
+    stream = torch.cuda.current_stream(device)
+    h_in = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t, _ in step.inputs()]
+    h_out = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t, _ in step.outputs()]
+    for d, h in h_in:
+        h.copy_(d)
+    h2d = sum(h.numel() * h.element_size() for _, h in h_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in h_out)
+
+    def one():
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        step.run()
+        for d, h in h_out:
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    barrier()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    return start.elapsed_time(end), h2d, d2h
+
+
+# ------------------------------------------------------------ CPU oracle
+
+class OracleRunner:
+    """The CPU oracle over a row sample of the workload (the same four ops)."""
+
+    def __init__(self, w: W.Workload, host: dict):
+        import oracle
+        from oracle import build as obuild
+        obuild.build()
+        self.o = oracle
+        self.w = w
+        bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+        rv = W.rows_view
+        self.q, self.k = bits(rv(host["qk"]["q"])), bits(rv(host["qk"]["k"]))
+        self.wq, self.wk = bits(host["qk"]["q_weight"]), bits(host["qk"]["k_weight"])
+        self.ax = bits(rv(host["adaln"]["x"]))
+        self.mod = np.ascontiguousarray(bits(host["adaln"]["mod"]).reshape(-1))
+        self.rx, self.ry = bits(rv(host["res"]["x"])), bits(rv(host["res"]["y"]))
+        self.ab = bits(rv(host["swiglu"]["ab"]))
+        self.outs = {"q": np.empty_like(self.q), "k": np.empty_like(self.k), "a": np.empty_like(self.ax),
+                     "r": np.empty_like(self.rx),
+                     "s": np.empty((self.ab.shape[0], w.inner), dtype=np.uint16)}
+
+    def threads(self) -> int:
+        return self.o.num_threads()
+
+    def run(self, rows: np.ndarray) -> float:
+        """Seconds the four oracle calls take on ``rows``."""
+        w, o, C = self.w, self.o, self.w.hidden
+        t0 = time.perf_counter()
+        o.qk_rmsnorm_rope(self.q, self.k, self.wq, self.wk, w.cu_seqlens, w.cu_seqlens_padded,
+                          num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
+                          rope_grid=w.rope_grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
+                          rows=rows, q_out=self.outs["q"], k_out=self.outs["k"])
+        o.adaln_modulate(self.ax, self.mod, self.mod[C:], w.cu_seqlens, w.cu_seqlens_padded, hidden=C,
+                         eps=w.eps, mod_seq_stride=6 * C, rows=rows, out=self.outs["a"])
+        o.gated_residual(self.rx, self.ry, self.mod[2 * C:], w.cu_seqlens, w.cu_seqlens_padded, hidden=C,
+                         gate_seq_stride=6 * C, rows=rows, out=self.outs["r"])
+        o.swiglu(self.ab, self.ab.reshape(-1)[w.inner:], w.cu_seqlens, w.cu_seqlens_padded, inner=w.inner,
+                 a_row_stride=2 * w.inner, b_row_stride=2 * w.inner, nrows=self.ab.shape[0], rows=rows,
+                 out=self.outs["s"])
+        return time.perf_counter() - t0
+
+    def sample(self, n: int, seed: int) -> np.ndarray:
+        valid = self.w.valid_rows()
+        rng = np.random.default_rng(seed)
+        return np.sort(rng.choice(valid, size=min(n, valid.size), replace=False))
+
+    def calibrate(self, budget_s: float, seed: int = 7) -> int:
+        """Rows per sample so that one sample takes about budget_s."""
+        n = 64
+        t = self.run(self.sample(n, seed))
+        while t < 0.25 and n < self.w.num_valid:
+            n *= 4
+            t = self.run(self.sample(n, seed))
+        return int(max(16, min(self.w.num_valid, n * budget_s / max(t, 1e-6))))
+
+
+def cpu_baseline(w: W.Workload, host: dict, budget_s: float = 12.0) -> dict:
+    runner = OracleRunner(w, host)
+    n = runner.calibrate(budget_s)
+    rows = runner.sample(n, seed=11)
+    t = runner.run(rows)
+    return {"value": rows.size / t, "unit": UNIT, "cores": runner.threads(), "kind": "oracle",
+            "sample": f"{rows.size} of {w.num_valid} valid tokens of {w.name} (seeded random rows), "
+                      f"all four ops per token, fp64 C oracle, {t:.1f} s"}
+
+
+# ------------------------------------------------------------ main
+
+def config_block(w: W.Workload, n: int) -> dict:
+    return {"workload": w.name, "num_seqs": w.num_seqs, "valid_tokens": w.num_valid,
+            "padded_rows": w.num_rows_padded, "lengths": list(w.lengths), "hidden": w.hidden,
+            "heads": f"{w.num_q_heads}+{w.num_k_heads}x{w.head_dim}", "inner": w.inner,
+            "rope": "3d t/h/w 44/42/42 on 24x42 frames + 1d tail" if w.grids else "1d",
+            "ops_per_step": list(OPS),
+            "l2": "inputs larger than L2 (each op moves >= 1.4 GB per step vs 126 MB L2)",
+            "parallelism": f"dp{n}: every GPU runs its own batch, no collective on the data path"}
+
+
+def run_dit(args):
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from dit_token_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier()
+    w0 = W.workload(args.workload, args.seed)
+    w = dataclasses.replace(w0, seed=data_seed(args.seed, rank))
+    host = host_inputs(w)
+    step = Step(w, host, device)
+    sampler = ClockSampler(local)
+    sampler.start()
+    elapsed_ms, op_ms, (h0, h1) = time_device(step, args.steps, args.warmup, device)
+    sampler.stop()
+    clocks = sampler.summary(h0, h1)
+    max_ms = reduce_max(elapsed_ms, device)
+    op_ms_max = {op: reduce_max(v, device) for op, v in op_ms.items()}
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e2e_ms, h2d, d2h = time_e2e(step, e2e_steps, min(args.warmup, 3), device)
+    e2e_max = reduce_max(e2e_ms, device)
+
+    tokens = w.num_valid * world
+    value = tokens * args.steps / (max_ms / 1e3)
+    abytes = algorithmic_bytes(w)
+    peak, peak_kind = measured_peak()
+    ops = {}
+    for op in OPS:
+        gbs = abytes[op] / (op_ms_max[op] / 1e3) / 1e9
+        ops[op] = {"us": round(op_ms_max[op] * 1e3, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                   "bytes": abytes[op]}
+    dom = max(OPS, key=lambda o: op_ms_max[o])
+    dom_gbs = abytes[dom] / (op_ms_max[dom] / 1e3) / 1e9
+    step_gbs = sum(abytes.values()) / (max_ms / args.steps / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, 1+N(0,0.02) norm weights, N(0,0.1) modulation)",
+        "config": config_block(w, world),
+        "step_gbs": round(step_gbs, 1), "step_hbm_frac": round(step_gbs / peak, 4),
+        "ops": ops,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth", "unit": "GB/s",
+                     "frac": round(dom_gbs / peak, 4), "traffic": profiled_traffic(dom, w.name),
+                     "algorithmic_bytes": abytes[dom]},
+        "gpu_launches": len(OPS) * args.steps,
+        "e2e": {"value": round(tokens * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, host, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return  # the CPU oracle runs once, on rank 0
+    w = W.workload(args.workload, args.seed)
+    host = host_inputs(w)
+    runner = OracleRunner(w, host)
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    n = runner.calibrate(per_step)
+    for i in range(args.warmup):
+        runner.run(runner.sample(n, seed=100 + i))
+    times = [runner.run(runner.sample(n, seed=1000 + i)) for i in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    sample = (f"each step: {n} of {w.num_valid} valid tokens of {w.name} (seeded random rows), all four ops "
+              f"per token, fp64 C oracle")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(w, 1), "impl": "reference",
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": runner.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("dit", "reference"), default="dit")
+    ap.add_argument("--workload", default="batched_varlen", choices=W.WORKLOAD_NAMES)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, _, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_dit(args)
+
+
+if __name__ == "__main__":
+    main()

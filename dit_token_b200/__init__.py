@@ -1,1 +1,233 @@
-"""Fused per-token operators of a packed audio-video DiT block for B200."""
+"""Fused per-token operators of a packed audio-video DiT block, for B200.
+
+Python binding of the C ABI in ``include/dit_token.h`` (``libdit_token.so``,
+built in-tree by ``python -m dit_token_b200.build``).  Each function has the
+name of its C entry point and only marshals arguments: it reads pointers,
+row strides and the current CUDA stream from torch tensors and calls the
+library through ctypes.  Every step of the computation runs in the CUDA
+kernels; there is no CPU or PyTorch fallback -- a missing library raises.
+
+The operators (see the header for the exact definitions):
+
+* ``dit_qk_rmsnorm_rope``  per-head Q/K RMSNorm fused with 1D / 3D RoPE, in place
+* ``dit_adaln_modulate``   LN(x) * (1 + scale_b) + shift_b
+* ``dit_gated_residual``   x + gate_b * y
+* ``dit_swiglu``           silu(a) * b
+
+All run over a packed sequence described by ``cu_seqlens`` (cumulative valid
+lengths) and ``cu_seqlens_padded`` (row offsets), touching valid rows only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = ["dit_qk_rmsnorm_rope", "dit_adaln_modulate", "dit_gated_residual", "dit_swiglu",
+           "dit_validate_seqlens", "DitError", "library", "LIB_PATH", "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_token.so")
+
+STATUS = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_ALIGN",
+          4: "DIT_ERR_UNSUPPORTED", 5: "DIT_ERR_SEQLENS", 6: "DIT_ERR_CUDA"}
+
+
+class DitError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        super().__init__(f"{func}: {message} (status {status})")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_VP = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_F32 = ctypes.c_float
+
+_SIGNATURES = {
+    "dit_qk_rmsnorm_rope": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
+                            _VP, _I32, _I32, _I32, _F32, _F32, _VP],
+    "dit_adaln_modulate": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _VP],
+    "dit_gated_residual": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
+    "dit_swiglu": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
+    "dit_validate_seqlens": [_VP, _VP, _I32, _I64, _VP, _VP],
+    "dit_status_string": [_I32],
+    "dit_last_cuda_error": [],
+    "dit_abi_version": [],
+}
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libdit_token.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m dit_token_b200.build` "
+                               "(the operators have no fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_char_p if name == "dit_status_string" else ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def _call(name: str, *args) -> None:
+    L = library()
+    st = getattr(L, name)(*args)
+    if st != 0:
+        msg = L.dit_status_string(st).decode()
+        if st == 6:
+            msg += f" (cudaError {L.dit_last_cuda_error()})"
+        raise DitError(name, st, msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _rows(t: torch.Tensor, what: str) -> tuple:
+    """(pointer, row stride in elements) of a bf16 CUDA tensor whose first axis
+    is the padded row and whose remaining axes are contiguous."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{what}: expected bfloat16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{what}: expected a CUDA tensor")
+    if t.dim() < 2:
+        raise ValueError(f"{what}: expected [rows, ...]")
+    expect = 1
+    for d in range(t.dim() - 1, 0, -1):
+        if t.size(d) != 1 and t.stride(d) != expect:
+            raise ValueError(f"{what}: the per-row axes must be contiguous")
+        expect *= t.size(d)
+    return t.data_ptr(), t.stride(0)
+
+
+def _vec(t: torch.Tensor, what: str) -> int:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{what}: expected a bfloat16 CUDA tensor")
+    return t.data_ptr()
+
+
+def _seq_vectors(t: torch.Tensor, hidden: int, what: str) -> tuple:
+    """(pointer, per-sequence stride) of per-sequence vectors [num_seqs, hidden]
+    (any sequence stride, contiguous last axis)."""
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{what}: expected a bfloat16 CUDA tensor")
+    if t.dim() != 2 or t.size(1) != hidden or (t.stride(1) != 1 and hidden > 1):
+        raise ValueError(f"{what}: expected [num_seqs, {hidden}] with a contiguous last axis")
+    return t.data_ptr(), t.stride(0)
+
+
+def _packing(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor):
+    for t, n in ((cu_seqlens, "cu_seqlens"), (cu_seqlens_padded, "cu_seqlens_padded")):
+        if t.dtype != torch.int32 or not t.is_cuda or t.dim() != 1 or not t.is_contiguous():
+            raise TypeError(f"{n}: expected a contiguous int32 CUDA vector")
+    if cu_seqlens.numel() != cu_seqlens_padded.numel() or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens and cu_seqlens_padded must both have num_seqs + 1 entries")
+    return cu_seqlens.data_ptr(), cu_seqlens_padded.data_ptr(), cu_seqlens.numel() - 1
+
+
+def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor, k_weight: torch.Tensor,
+                        cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, *,
+                        num_q_heads: int, num_k_heads: int, head_dim: int,
+                        rope_grid: Optional[torch.Tensor] = None,
+                        sections: Sequence[int] = (0, 0, 0), rope_theta: float = 10000.0,
+                        eps: float = 1e-6, stream=None) -> None:
+    """In place: q, k <- RoPE(RMSNorm_head(q) * q_weight), RoPE(RMSNorm_head(k) * k_weight).
+
+    q: [rows, num_q_heads * head_dim] (or [rows, heads, head_dim]) bf16, any
+    row stride; k likewise.  rope_grid: int32 [num_seqs, 3] (T, H, W) or None
+    (every row 1D); sections: t/h/w widths of head_dim on 3D rows."""
+    qp, qs = _rows(q, "q")
+    kp, ks = _rows(k, "k")
+    if k.size(0) != q.size(0):
+        raise ValueError("q and k must have the same number of rows")
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    gp = 0
+    if rope_grid is not None:
+        if rope_grid.dtype != torch.int32 or not rope_grid.is_cuda or not rope_grid.is_contiguous() \
+                or tuple(rope_grid.shape) != (B, 3):
+            raise TypeError("rope_grid: expected a contiguous int32 CUDA tensor [num_seqs, 3]")
+        gp = rope_grid.data_ptr()
+    st, sh, sw = (int(s) for s in sections)
+    _call("dit_qk_rmsnorm_rope", qp, qs, kp, ks, _vec(q_weight, "q_weight"), _vec(k_weight, "k_weight"),
+          cs, cp, B, q.size(0), num_q_heads, num_k_heads, head_dim, gp or None, st, sh, sw,
+          float(rope_theta), float(eps), _stream(stream))
+
+
+def dit_adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
+                       cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, *,
+                       out: Optional[torch.Tensor] = None, eps: float = 1e-6, stream=None) -> torch.Tensor:
+    """out = LayerNorm(x) * (1 + scale_b) + shift_b on valid rows.
+
+    x: [rows, hidden]; shift, scale: [num_seqs, hidden] (any sequence stride,
+    e.g. slices of a [num_seqs, 6, hidden] modulation tensor -- both must
+    share it).  ``out`` may be x; if None a new tensor is returned whose
+    padding rows are left uninitialised."""
+    hidden = x.size(-1)
+    if out is None:
+        out = torch.empty_like(x)
+    xp, xs = _rows(x, "x")
+    op, os_ = _rows(out, "out")
+    shp, sst = _seq_vectors(shift, hidden, "shift")
+    scp, cst = _seq_vectors(scale, hidden, "scale")
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    if B > 1 and sst != cst:
+        raise ValueError("shift and scale must share one sequence stride")
+    _call("dit_adaln_modulate", xp, xs, op, os_, shp, scp, sst if B > 1 else hidden, cs, cp, B, x.size(0),
+          hidden, float(eps), _stream(stream))
+    return out
+
+
+def dit_gated_residual(x: torch.Tensor, y: torch.Tensor, gate: torch.Tensor,
+                       cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, *,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out = x + gate_b * y on valid rows (``out`` may be x)."""
+    hidden = x.size(-1)
+    if out is None:
+        out = torch.empty_like(x)
+    xp, xs = _rows(x, "x")
+    yp, ys = _rows(y, "y")
+    op, os_ = _rows(out, "out")
+    gp, gst = _seq_vectors(gate, hidden, "gate")
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    _call("dit_gated_residual", xp, xs, yp, ys, gp, gst if B > 1 else hidden, op, os_, cs, cp, B,
+          x.size(0), hidden, _stream(stream))
+    return out
+
+
+def dit_swiglu(a: torch.Tensor, b: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor,
+               *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out = silu(a) * b on valid rows.  a, b: [rows, inner] (e.g. the two
+    column halves of a [rows, 2 * inner] projection)."""
+    inner = a.size(-1)
+    if b.size(-1) != inner:
+        raise ValueError("a and b must have the same width")
+    if out is None:
+        out = torch.empty((a.size(0), inner), dtype=a.dtype, device=a.device)
+    ap, as_ = _rows(a, "a")
+    bp, bs = _rows(b, "b")
+    op, os_ = _rows(out, "out")
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    _call("dit_swiglu", ap, as_, bp, bs, op, os_, cs, cp, B, a.size(0), inner, _stream(stream))
+    return out
+
+
+def dit_validate_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, num_rows_padded: int,
+                         *, flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Enqueue the device-side descriptor check; returns the int32[2] flag
+    tensor (flag[0] == 1: malformed, flag[1]: first bad sequence)."""
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    if flag is None:
+        flag = torch.empty(2, dtype=torch.int32, device=cu_seqlens.device)
+    _call("dit_validate_seqlens", cs, cp, B, int(num_rows_padded), flag.data_ptr(), _stream(stream))
+    return flag

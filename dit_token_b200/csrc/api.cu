@@ -1,0 +1,233 @@
+// api.cu -- the C ABI declared in include/dit_token.h: host-side argument
+// checks, the per-pair rotary frequency tables, and the launches.  Nothing
+// here allocates, synchronizes or keeps state beyond a thread-local copy of
+// the last CUDA error.
+#include <cmath>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "dit_token.h"
+#include "launch.h"
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool mult8(int64_t v) { return (v & 7) == 0; }
+
+dit_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return DIT_OK;
+    g_last_cuda_error = (int32_t)e;
+    return DIT_ERR_CUDA;
+}
+
+// Checks shared by every operator: sizes, then the descriptor pointers.
+// Returns DIT_OK and sets *nothing_to_do when the batch is empty.
+dit_status check_packing(const int32_t* cs, const int32_t* cp, int32_t num_seqs, int64_t num_rows_padded,
+                         bool* nothing_to_do)
+{
+    if (num_seqs < 0 || num_rows_padded < 0 || num_rows_padded > INT32_MAX)
+        return DIT_ERR_SHAPE;
+    *nothing_to_do = (num_seqs == 0 || num_rows_padded == 0);
+    if (*nothing_to_do)
+        return DIT_OK;
+    if (!cs || !cp)
+        return DIT_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(cs) & 3u) || (reinterpret_cast<uintptr_t>(cp) & 3u))
+        return DIT_ERR_ALIGN;
+    return DIT_OK;
+}
+
+dit::Packing packing(const int32_t* cs, const int32_t* cp, int32_t num_seqs, int64_t num_rows_padded)
+{
+    return dit::Packing{cs, cp, num_seqs, (int32_t)num_rows_padded};
+}
+
+}  // namespace
+
+extern "C" {
+
+dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                               const void* q_weight, const void* k_weight,
+                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                               int32_t num_seqs, int64_t num_rows_padded,
+                               int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+                               const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+                               float rope_theta, float eps, void* stream)
+{
+    bool empty = false;
+    dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
+    if (st != DIT_OK)
+        return st;
+    if (num_q_heads < 0 || num_k_heads < 0 || head_dim <= 0)
+        return DIT_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128)
+        return DIT_ERR_UNSUPPORTED;
+    if (q_row_stride < (int64_t)num_q_heads * head_dim || k_row_stride < (int64_t)num_k_heads * head_dim)
+        return DIT_ERR_SHAPE;
+    if (!(rope_theta > 0.f) || !(eps >= 0.f) || !std::isfinite(rope_theta) || !std::isfinite(eps))
+        return DIT_ERR_SHAPE;
+    if (rope_grid) {
+        if (sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t | sec_h | sec_w) & 1 ||
+            (int64_t)sec_t + sec_h + sec_w != head_dim)
+            return DIT_ERR_SHAPE;
+    }
+    if (empty || num_q_heads + num_k_heads == 0)
+        return DIT_OK;
+    if (!q || !k || !q_weight || !k_weight)
+        return DIT_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_weight) || !aligned16(k_weight) ||
+        !mult8(q_row_stride) || !mult8(k_row_stride) ||
+        (rope_grid && (reinterpret_cast<uintptr_t>(rope_grid) & 3u)))
+        return DIT_ERR_ALIGN;
+
+    dit::QkParams p{};
+    p.q = static_cast<uint16_t*>(q);
+    p.k = static_cast<uint16_t*>(k);
+    p.q_weight = static_cast<const uint16_t*>(q_weight);
+    p.k_weight = static_cast<const uint16_t*>(k_weight);
+    p.rope_grid = rope_grid;
+    p.q_row_stride = q_row_stride;
+    p.k_row_stride = k_row_stride;
+    p.pk = packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded);
+    p.num_q_heads = num_q_heads;
+    p.num_k_heads = num_k_heads;
+    p.eps = eps;
+    // Rotary frequencies in fp64: theta^(-2j/D) for 1D rows; on 3D rows pair j
+    // belongs to the t, h or w section and uses theta^(-2j'/d_s) with j' its
+    // index inside that section of width d_s.
+    const double theta = (double)rope_theta;
+    const int pairs = head_dim / 2;
+    const int sec[3] = {sec_t, sec_h, sec_w};
+    for (int j = 0; j < pairs; ++j) {
+        p.inv_freq_1d[j] = std::pow(theta, -2.0 * j / head_dim);
+        int first = 0, axis = 2;
+        for (int s = 0; s < 3; ++s) {
+            if (j < first + sec[s] / 2) {
+                axis = s;
+                break;
+            }
+            first += sec[s] / 2;
+        }
+        p.axis[j] = (int8_t)axis;
+        p.inv_freq_3d[j] = rope_grid ? std::pow(theta, -2.0 * (j - first) / sec[axis]) : 0.0;
+    }
+    return from_cuda(dit::launch_qk_rmsnorm_rope(p, head_dim, static_cast<cudaStream_t>(stream)));
+}
+
+dit_status dit_adaln_modulate(const void* x, int64_t x_row_stride, void* out, int64_t out_row_stride,
+                              const void* shift, const void* scale, int64_t mod_seq_stride,
+                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                              int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
+                              void* stream)
+{
+    bool empty = false;
+    dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
+    if (st != DIT_OK)
+        return st;
+    if (hidden <= 0 || x_row_stride < hidden || out_row_stride < hidden || mod_seq_stride < 0 ||
+        !(eps >= 0.f) || !std::isfinite(eps))
+        return DIT_ERR_SHAPE;
+    if (hidden > dit::kMaxAdalnHidden)
+        return DIT_ERR_UNSUPPORTED;
+    if (empty)
+        return DIT_OK;
+    if (!x || !out || !shift || !scale)
+        return DIT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(shift) || !aligned16(scale) || !mult8(hidden) ||
+        !mult8(x_row_stride) || !mult8(out_row_stride) || !mult8(mod_seq_stride))
+        return DIT_ERR_ALIGN;
+    dit::AdalnParams p{static_cast<const uint16_t*>(x), static_cast<uint16_t*>(out),
+                       static_cast<const uint16_t*>(shift), static_cast<const uint16_t*>(scale),
+                       x_row_stride, out_row_stride, mod_seq_stride,
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps};
+    return from_cuda(dit::launch_adaln_modulate(p, static_cast<cudaStream_t>(stream)));
+}
+
+dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                              const void* gate, int64_t gate_seq_stride, void* out, int64_t out_row_stride,
+                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                              int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, void* stream)
+{
+    bool empty = false;
+    dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
+    if (st != DIT_OK)
+        return st;
+    if (hidden <= 0 || x_row_stride < hidden || y_row_stride < hidden || out_row_stride < hidden ||
+        gate_seq_stride < 0)
+        return DIT_ERR_SHAPE;
+    if (empty)
+        return DIT_OK;
+    if (!x || !y || !gate || !out)
+        return DIT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(gate) || !aligned16(out) || !mult8(hidden) ||
+        !mult8(x_row_stride) || !mult8(y_row_stride) || !mult8(out_row_stride) || !mult8(gate_seq_stride))
+        return DIT_ERR_ALIGN;
+    dit::GatedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y),
+                       static_cast<const uint16_t*>(gate), static_cast<uint16_t*>(out),
+                       x_row_stride, y_row_stride, gate_seq_stride, out_row_stride,
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden};
+    return from_cuda(dit::launch_gated_residual(p, static_cast<cudaStream_t>(stream)));
+}
+
+dit_status dit_swiglu(const void* a, int64_t a_row_stride, const void* b, int64_t b_row_stride,
+                      void* out, int64_t out_row_stride,
+                      const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                      int32_t num_seqs, int64_t num_rows_padded, int32_t inner, void* stream)
+{
+    bool empty = false;
+    dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
+    if (st != DIT_OK)
+        return st;
+    if (inner <= 0 || a_row_stride < inner || b_row_stride < inner || out_row_stride < inner)
+        return DIT_ERR_SHAPE;
+    if (empty)
+        return DIT_OK;
+    if (!a || !b || !out)
+        return DIT_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(out) || !mult8(inner) || !mult8(a_row_stride) ||
+        !mult8(b_row_stride) || !mult8(out_row_stride))
+        return DIT_ERR_ALIGN;
+    dit::SwigluParams p{static_cast<const uint16_t*>(a), static_cast<const uint16_t*>(b),
+                        static_cast<uint16_t*>(out), a_row_stride, b_row_stride, out_row_stride,
+                        packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), inner};
+    return from_cuda(dit::launch_swiglu(p, static_cast<cudaStream_t>(stream)));
+}
+
+dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                int32_t num_seqs, int64_t num_rows_padded, int32_t* flag, void* stream)
+{
+    if (num_seqs < 0 || num_rows_padded < 0 || num_rows_padded > INT32_MAX)
+        return DIT_ERR_SHAPE;
+    if (!cu_seqlens || !cu_seqlens_padded || !flag)
+        return DIT_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_padded) & 3u) ||
+        (reinterpret_cast<uintptr_t>(flag) & 3u))
+        return DIT_ERR_ALIGN;
+    dit::Packing pk = packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded);
+    return from_cuda(dit::launch_validate_seqlens(pk, num_rows_padded, flag, static_cast<cudaStream_t>(stream)));
+}
+
+const char* dit_status_string(dit_status s)
+{
+    switch (s) {
+    case DIT_OK: return "DIT_OK";
+    case DIT_ERR_NULL: return "DIT_ERR_NULL: a required pointer is NULL";
+    case DIT_ERR_SHAPE: return "DIT_ERR_SHAPE: invalid size, stride or rope sections";
+    case DIT_ERR_ALIGN: return "DIT_ERR_ALIGN: pointer not 16-byte aligned or size/stride not a multiple of 8";
+    case DIT_ERR_UNSUPPORTED: return "DIT_ERR_UNSUPPORTED: unsupported head_dim or hidden size";
+    case DIT_ERR_SEQLENS: return "DIT_ERR_SEQLENS: malformed cu_seqlens / cu_seqlens_padded";
+    case DIT_ERR_CUDA: return "DIT_ERR_CUDA: kernel launch failed";
+    default: return "unknown dit_status";
+    }
+}
+
+int32_t dit_last_cuda_error(void) { return g_last_cuda_error; }
+
+int32_t dit_abi_version(void) { return DIT_ABI_VERSION; }
+
+}  // extern "C"

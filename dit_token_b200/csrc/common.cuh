@@ -1,0 +1,134 @@
+// common.cuh -- device helpers shared by the fused DiT token kernels:
+// packed-row mapping, 128-bit bf16 vector I/O and bf16 <-> fp32 conversion.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dit {
+
+constexpr int kWarp = 32;
+constexpr int kCtaThreads = 256;          // 8 warps
+constexpr int kWarpsPerCta = kCtaThreads / kWarp;
+
+// ------------------------------------------------------------ packed rows
+//
+// The packed batch holds num_seqs sequences; sequence b owns padded rows
+// [cp[b], cp[b+1]) and its first cs[b+1] - cs[b] rows are valid.  Work is
+// indexed by the VALID-row ordinal v in [0, cs[B]) so that padding costs no
+// thread: v lives in sequence b = max{b : cs[b] <= v} at padded row
+// cp[b] + (v - cs[b]).  "Why Real-Time MiniMax H3 Serving Requires More Than
+// a Faster DiT", "Key takeaways", bullet 1: work follows each sequence's
+// valid length, so the padding rows at its end cost nothing.
+
+struct RowSlot {
+    int32_t row;    // padded row index
+    int32_t seq;    // sequence index b
+    int32_t local;  // index of the row within its sequence (RoPE position)
+};
+
+// Largest b in [0, B) with cs[b] <= v, or -1.  Warp-collective (every lane
+// passes the same v): a 32-way search, one ballot per level, so B <= 32 costs
+// a single round of loads and B <= 1024 two.
+__device__ __forceinline__ int find_seq(int v, const int32_t* __restrict__ cs, int B, int lane)
+{
+    int lo = 0, n = B;
+    while (n > kWarp) {
+        const int step = (n + kWarp - 1) / kWarp;
+        const int idx = lane * step;
+        const bool ok = idx < n && __ldg(cs + lo + idx) <= v;
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        if (m == 0u)
+            return -1;
+        const int kk = 31 - __clz(m);
+        lo += kk * step;
+        n = min(step, n - kk * step);
+    }
+    const bool ok = lane < n && __ldg(cs + lo + lane) <= v;
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    return m == 0u ? -1 : lo + 31 - __clz(m);
+}
+
+// Maps valid-row ordinal v to its padded row.  Warp-collective; returns false
+// (for the whole warp) when v is past the last valid row or when the device
+// descriptor points outside the buffer -- such rows are skipped, never
+// followed out of bounds.
+__device__ __forceinline__ bool map_valid_row(int v, const int32_t* __restrict__ cs,
+                                              const int32_t* __restrict__ cp, int B,
+                                              int rows_padded, int lane, RowSlot& s)
+{
+    const int b = find_seq(v, cs, B, lane);
+    if (b < 0)
+        return false;
+    const int cs0 = __ldg(cs + b), cs1 = __ldg(cs + b + 1);
+    const int cp0 = __ldg(cp + b), cp1 = __ldg(cp + b + 1);
+    const int r = v - cs0;
+    if (r < 0 || r >= cs1 - cs0 || r >= cp1 - cp0)
+        return false;
+    const long long row = (long long)cp0 + r;
+    if (row < 0 || row >= rows_padded)
+        return false;
+    s.row = (int32_t)row;
+    s.seq = b;
+    s.local = r;
+    return true;
+}
+
+// ---------------------------------------------------------- vector I/O
+// Streamed activations are touched once: load and store them with the
+// evict-first (".cs") policy so they do not push the small per-sequence
+// vectors (gates, shifts, scales, norm weights) out of L2.  Those go through
+// the read-only path (__ldg) instead.
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p)
+{
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void st_stream(uint16_t* p, uint4 v)
+{
+    __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
+__device__ __forceinline__ uint4 ld_shared_vec(const uint16_t* p)
+{
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// ------------------------------------------------------ bf16 <-> fp32
+// A bf16 value is the upper half of a binary32 value, so widening is a shift.
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
+{
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+    f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// Two fp32 values -> one bf16x2 word (round to nearest, ties to even).
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8])
+{
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float v)
+{
+#pragma unroll
+    for (int o = WIDTH / 2; o >= 1; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace dit

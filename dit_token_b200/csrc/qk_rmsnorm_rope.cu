@@ -1,0 +1,141 @@
+// qk_rmsnorm_rope.cu -- per-head RMSNorm of q and k fused with rotary position
+// embedding, in place, over the valid rows of a packed sequence ("Why
+// Real-Time MiniMax H3 Serving Requires More Than a Faster DiT", "Key
+// takeaways", bullet 2: the Q/K normalization is fused with the rotary
+// embedding; bullet 1: rotary rows are computed only where needed).
+//
+// Layout.  One warp per valid row.  A head of D = 8*LPH elements is held by a
+// group of LPH lanes, 8 elements (one 16-byte vector) per lane, so the
+// per-head sum of squares is a log2(LPH)-step xor-shuffle reduction and every
+// lane owns 4 complete interleaved pairs (2j, 2j+1): the rotation is
+// lane-local.  A lane always sits at the same offset inside a head, so it
+// needs the cos/sin of only its own 4 pairs: it computes them once per row
+// (angle reduced in fp64, then sincosf) and reuses them for all
+// num_q_heads + num_k_heads heads of that row -- cos/sin are never re-read or
+// recomputed per head.  Each step issues U head vectors per lane before any
+// arithmetic.  HBM traffic: q and k are each read once and written once, 4
+// bytes per element.
+#include "common.cuh"
+#include "launch.h"
+
+namespace dit {
+namespace {
+
+constexpr int kUnroll = 4;
+
+// angle mod 2*pi in fp64, then single precision: keeps the angle exact to
+// ~1e-7 rad for any position, and lets sincosf take its short path.
+__device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
+{
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+    const double red = angle - kTwoPi * rint(angle * kInvTwoPi);
+    sincosf((float)red, &s, &c);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCtaThreads)
+qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
+{
+    constexpr int LPH = D / 8;          // lanes per head
+    constexpr int HPW = kWarp / LPH;    // heads per warp per step
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    RowSlot s;
+    if (!map_valid_row(v, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs,
+                       p.pk.num_rows_padded, lane, s))
+        return;
+    const int sub = lane / LPH;  // which head of the step
+    const int li = lane % LPH;   // position inside the head: elements 8*li .. 8*li+7
+
+    // Positions of this row: a row inside the sequence's T x H x W video grid
+    // (t-major, then h, then w) is 3D; every later row is 1D, counted from the
+    // end of the grid.  Without a grid every row is 1D.
+    bool is3d = false;
+    long long pt = 0, ph = 0, pw = 0;
+    long long pos1 = s.local;
+    if (p.rope_grid != nullptr) {
+        const long long T = __ldg(p.rope_grid + 3 * s.seq);
+        const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
+        const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
+        const long long thw = T * H * W;
+        if (s.local < thw) {
+            is3d = true;
+            pt = s.local / (H * W);
+            ph = (s.local / W) % H;
+            pw = s.local % W;
+        } else {
+            pos1 = s.local - thw;
+        }
+    }
+    float cs[4], sn[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int j = 4 * li + e;
+        const int ax = p.axis[j];
+        const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
+        const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
+        pair_cos_sin(ang, cs[e], sn[e]);
+    }
+    float wq[8], wk[8];
+    unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
+    unpack8(ld_shared_vec(p.k_weight + 8 * li), wk);
+
+    const int Hq = p.num_q_heads;
+    const int Htot = Hq + p.num_k_heads;
+    uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride + 8 * li;
+    uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride + 8 * li;
+    const float inv_d = 1.0f / (float)D;
+
+    for (int h0 = 0; h0 < Htot; h0 += HPW * kUnroll) {
+        uint4 xv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int h = h0 + u * HPW + sub;
+            if (h < Htot)
+                xv[u] = ld_stream(h < Hq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D);
+            else
+                xv[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int h = h0 + u * HPW + sub;
+            float x[8];
+            unpack8(xv[u], x);
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                ss = fmaf(x[e], x[e], ss);
+            ss = group_sum<LPH>(ss);  // every lane of the warp takes part
+            if (h < Htot) {
+                const float r = rsqrtf(ss * inv_d + p.eps);
+                const bool isq = h < Hq;
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float y0 = x[2 * e] * r * (isq ? wq[2 * e] : wk[2 * e]);
+                    const float y1 = x[2 * e + 1] * r * (isq ? wq[2 * e + 1] : wk[2 * e + 1]);
+                    o[2 * e] = y0 * cs[e] - y1 * sn[e];
+                    o[2 * e + 1] = y0 * sn[e] + y1 * cs[e];
+                }
+                st_stream(isq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D, pack8(o));
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, cudaStream_t stream)
+{
+    const unsigned grid = (unsigned)((p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta);
+    if (head_dim == 128)
+        qk_rmsnorm_rope_kernel<128><<<grid, kCtaThreads, 0, stream>>>(p);
+    else if (head_dim == 64)
+        qk_rmsnorm_rope_kernel<64><<<grid, kCtaThreads, 0, stream>>>(p);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace dit

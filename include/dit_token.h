@@ -1,0 +1,176 @@
+/*
+ * dit_token.h -- C ABI of the fused per-token operators of a packed
+ * audio-video diffusion-transformer (DiT) block, for NVIDIA B200 (sm_100a).
+ *
+ * The operators are the ones named in "Why Real-Time MiniMax H3 Serving
+ * Requires More Than a Faster DiT", section "Key takeaways", bullet 2 (Q/K
+ * RMSNorm with RoPE, modulation and normalization, residual updates and
+ * SwiGLU, fused to cut repeated small launches) and in "MiniMax H3 通过
+ * vLLM-Omni 实现 FastH3 实时推理", section "vLLM-Omni 中的系统级优化",
+ * bullet 2.  They run over a packed sequence whose valid lengths come from
+ * cu_seqlens, so structural suffix padding is never touched (first page,
+ * "Key takeaways", bullet 1; third page, same section, bullet 1).  The pages
+ * print no formulas; each entry point states the standard definition it
+ * computes.
+ *
+ * Common conventions
+ * ------------------
+ * Data type   every activation, weight and modulation vector is bf16
+ *             (IEEE binary32 upper half), row-major; arithmetic is fp32 and
+ *             every output element is rounded once, to nearest-even.
+ * Pointers    all tensor pointers are DEVICE pointers, owned by the caller;
+ *             they must be 16-byte aligned.  Strides are in ELEMENTS and must
+ *             be multiples of 8 (16 bytes); so must hidden, inner and
+ *             head_dim.
+ * Packing     cu_seqlens[num_seqs+1] (device, int32): cumulative VALID lengths,
+ *             cu_seqlens[0] = 0.  cu_seqlens_padded[num_seqs+1] (device,
+ *             int32): first padded row of every sequence, the last entry the
+ *             end of the used rows (<= num_rows_padded).  Row
+ *             cu_seqlens_padded[b] + r is valid iff
+ *             r < cu_seqlens[b+1] - cu_seqlens[b]; every other row (suffix
+ *             padding) is neither read nor written.  The device arrays are
+ *             trusted but never followed out of bounds: a row index outside
+ *             [0, num_rows_padded) or past a sequence's padded slot is
+ *             skipped.  dit_validate_seqlens checks them on the device.
+ * Aliasing    in-place use is allowed only as exact aliasing (same pointer
+ *             and stride): out == x for dit_adaln_modulate and
+ *             dit_gated_residual; q and k are always updated in place.
+ *             Partial overlap is undefined.
+ * Stream      `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *             Calls only enqueue work: they never synchronize, allocate or
+ *             keep state, and are safe to call from several host threads.
+ * Errors      argument errors are returned BEFORE anything is launched; a
+ *             failed launch returns DIT_ERR_CUDA (dit_last_cuda_error gives
+ *             the CUDA error code seen by this thread).  No entry point traps
+ *             on the device.
+ */
+#ifndef DIT_TOKEN_H
+#define DIT_TOKEN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t dit_status;
+enum {
+    DIT_OK = 0,
+    DIT_ERR_NULL = 1,        /* a required pointer is NULL */
+    DIT_ERR_SHAPE = 2,       /* negative/zero size, stride too small, bad sections */
+    DIT_ERR_ALIGN = 3,       /* pointer not 16-byte aligned or size/stride not a multiple of 8 */
+    DIT_ERR_UNSUPPORTED = 4, /* e.g. head_dim other than 64 or 128 */
+    DIT_ERR_SEQLENS = 5,     /* dit_validate_seqlens found a malformed descriptor */
+    DIT_ERR_CUDA = 6         /* the kernel launch failed */
+};
+
+#define DIT_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DIT_API __attribute__((visibility("default")))
+#else
+#define DIT_API
+#endif
+
+/* Per-head Q/K RMSNorm fused with rotary position embedding (RoPE), in place.
+ *
+ * Pages: first page "Key takeaways" bullet 2 (the Q/K normalization fused
+ * with the rotary embedding) and bullet 1 (rotary rows are computed only for
+ * the rows a rank needs).  For every valid row and every head h of q (weight
+ * q_weight) and of k (weight k_weight):
+ *   ms   = (1/D) sum_i x_i^2
+ *   y_i  = x_i * rsqrt(ms + eps) * w_i
+ *   (o_2j, o_2j+1) = (y_2j c - y_2j+1 s, y_2j s + y_2j+1 c),  c, s = cos, sin(angle_j)
+ * with interleaved pairs (2j, 2j+1).  Angles:
+ *   rope_grid == NULL: angle_j = p * theta^(-2j/D), p = row index within its sequence;
+ *   rope_grid[b] = (T, H, W): rows r < T*H*W of sequence b are video latents at
+ *     (t, h, w) = (r / (H W), (r / W) mod H, r mod W); head_dim is split into
+ *     sections of sec_t, sec_h, sec_w elements (in that order) and pair j' of
+ *     the section of axis s (width d_s) turns by p_s * theta^(-2j'/d_s);
+ *     rows r >= T*H*W (audio) use the 1D angle with p = r - T*H*W.
+ *
+ * q            device bf16 [num_rows_padded][num_q_heads * head_dim], row stride q_row_stride
+ *              (>= num_q_heads * head_dim; may be a slice of a fused QKV buffer)
+ * k            likewise with num_k_heads (num_k_heads may differ from num_q_heads)
+ * q_weight     device bf16 [head_dim], shared by all q heads; k_weight likewise for k
+ * rope_grid    device int32 [num_seqs][3] or NULL
+ * sec_*        even, >= 0, summing to head_dim when rope_grid != NULL (ignored otherwise)
+ * head_dim     64 or 128 (else DIT_ERR_UNSUPPORTED)
+ */
+DIT_API dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                               const void* q_weight, const void* k_weight,
+                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                               int32_t num_seqs, int64_t num_rows_padded,
+                               int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+                               const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+                               float rope_theta, float eps, void* stream);
+
+/* Adaptive LayerNorm modulation: out = LN(x) * (1 + scale_b) + shift_b.
+ *
+ * Pages: first page "Key takeaways" bullet 2 (the modulation and the
+ * normalization are fused).  LN has no affine: mean and biased variance over the hidden axis,
+ * x_hat = (x - mean) * rsqrt(var + eps).  shift/scale are per sequence b.
+ *
+ * x, out       device bf16 [num_rows_padded][hidden], row strides >= hidden (out may be x)
+ * shift, scale device bf16, vector of sequence b at shift + b * mod_seq_stride
+ *              (mod_seq_stride >= 0, a multiple of 8; e.g. 6*hidden for a [B][6][hidden]
+ *              modulation tensor)
+ */
+DIT_API dit_status dit_adaln_modulate(const void* x, int64_t x_row_stride, void* out, int64_t out_row_stride,
+                              const void* shift, const void* scale, int64_t mod_seq_stride,
+                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                              int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
+                              void* stream);
+
+/* Gated residual update: out = x + gate_b * y (one fp32 fused multiply-add,
+ * one rounding).
+ *
+ * Pages: first page "Key takeaways" bullet 2 (the residual update is fused).
+ * x, y, out    device bf16 [num_rows_padded][hidden] with their own row strides (out may be x)
+ * gate         device bf16, vector of sequence b at gate + b * gate_seq_stride
+ */
+DIT_API dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                              const void* gate, int64_t gate_seq_stride, void* out, int64_t out_row_stride,
+                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                              int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, void* stream);
+
+/* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)).
+ *
+ * Pages: first page "Key takeaways" bullet 2 and third page "vLLM-Omni 中的
+ * 系统级优化" bullet 2 (the SwiGLU activation is fused).
+ * a, b         device bf16 [num_rows_padded][inner] with their own row strides; for a
+ *              chunked [rows][2*inner] projection pass a = base, b = base + inner and
+ *              both row strides 2*inner
+ * out          device bf16 [num_rows_padded][inner], row stride out_row_stride
+ */
+DIT_API dit_status dit_swiglu(const void* a, int64_t a_row_stride, const void* b, int64_t b_row_stride,
+                      void* out, int64_t out_row_stride,
+                      const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                      int32_t num_seqs, int64_t num_rows_padded, int32_t inner, void* stream);
+
+/* Device-side check of a packing descriptor; no counterpart on the pages (it
+ * guards the padding-free packing of the first page, "Key takeaways" bullet 1).
+ * Writes flag[0] = 0 if cu_seqlens[0] == 0, cu_seqlens_padded[0] == 0, both
+ * are non-decreasing, every valid length fits its padded slot and
+ * cu_seqlens_padded[num_seqs] <= num_rows_padded; otherwise flag[0] = 1 and
+ * flag[1] = the first offending sequence index.  flag: device int32[2].  The
+ * kernel never traps; the host reads the flag when it chooses to (e.g. with
+ * cudaMemcpy after the stream) and maps 1 to DIT_ERR_SEQLENS. */
+DIT_API dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                int32_t num_seqs, int64_t num_rows_padded, int32_t* flag, void* stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+DIT_API const char* dit_status_string(dit_status s);
+
+/* The CUDA error code (cudaError_t value) behind the last DIT_ERR_CUDA
+ * returned on the calling thread, 0 if none. */
+DIT_API int32_t dit_last_cuda_error(void);
+
+/* DIT_ABI_VERSION of the library. */
+DIT_API int32_t dit_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_TOKEN_H */

@@ -119,7 +119,7 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
                     num_q_heads, num_k_heads, head_dim, rope_grid=None,
                     sections=(0, 0, 0), rope_theta=10000.0, eps=1e-6,
                     q_row_stride=None, k_row_stride=None, rows=None,
-                    q_out_init=None, k_out_init=None, want_f64=False):
+                    q_out_init=None, k_out_init=None, want_f64=False, q_out=None, k_out=None):
     """Per-head Q/K RMSNorm fused with 1D / 3D rotary embedding.
 
     q, k: uint16 arrays whose first axis is the padded row; row strides
@@ -130,8 +130,10 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
     q, qs = _flat_view(q, q_row_stride, None)
     k, ks = _flat_view(k, k_row_stride, None)
     nrows = q.shape[0]
-    q_out = np.array(q if q_out_init is None else q_out_init, dtype=np.uint16, copy=True)
-    k_out = np.array(k if k_out_init is None else k_out_init, dtype=np.uint16, copy=True)
+    if q_out is None:
+        q_out = np.array(q if q_out_init is None else q_out_init, dtype=np.uint16, copy=True)
+    if k_out is None:
+        k_out = np.array(k if k_out_init is None else k_out_init, dtype=np.uint16, copy=True)
     q64 = np.full(q.shape, np.nan) if want_f64 else None
     k64 = np.full(k.shape, np.nan) if want_f64 else None
     grid = None if rope_grid is None else np.ascontiguousarray(np.asarray(rope_grid, dtype=np.int32))
@@ -156,7 +158,7 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
 
 def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
                    mod_seq_stride=None, x_row_stride=None, rows=None, out_init=None,
-                   want_f64=False):
+                   want_f64=False, out=None):
     """out = LayerNorm(x) * (1 + scale_b) + shift_b on valid rows.
 
     shift, scale: uint16 arrays [num_seqs, ...] read with mod_seq_stride
@@ -165,7 +167,8 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
     nrows = x.shape[0]
-    out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
+    if out is None:
+        out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
     o64 = np.full(out.shape, np.nan) if want_f64 else None
     sh = np.ascontiguousarray(_u16(shift))
     sc = np.ascontiguousarray(_u16(scale))
@@ -181,14 +184,15 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
 
 def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_seq_stride=None,
                    x_row_stride=None, y_row_stride=None, rows=None, out_init=None,
-                   want_f64=False):
+                   want_f64=False, out=None):
     """out = x + gate_b * y on valid rows."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
     y, ys = _flat_view(y, y_row_stride, None)
     nrows = x.shape[0]
-    out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
+    if out is None:
+        out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
     o64 = np.full(out.shape, np.nan) if want_f64 else None
     g = np.ascontiguousarray(_u16(gate))
     gss = hidden if gate_seq_stride is None else gate_seq_stride
@@ -202,7 +206,7 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
 
 
 def swiglu(a, b, cu_seqlens, cu_seqlens_padded, *, inner, a_row_stride=None, b_row_stride=None,
-           out_row_stride=None, nrows=None, rows=None, out_init=None, want_f64=False):
+           out_row_stride=None, nrows=None, rows=None, out_init=None, want_f64=False, out=None):
     """out = silu(a) * b on valid rows.
 
     a, b: uint16 arrays whose first axis is the padded row (for a chunked
@@ -215,7 +219,9 @@ def swiglu(a, b, cu_seqlens, cu_seqlens_padded, *, inner, a_row_stride=None, b_r
     b, bs = _flat_view(b, b_row_stride, None)
     n = a.shape[0] if nrows is None else nrows
     ostride = inner if out_row_stride is None else out_row_stride
-    if out_init is None:
+    if out is not None:
+        pass
+    elif out_init is None:
         out = np.full((n, ostride), 0x7FC1, dtype=np.uint16)
     else:
         out = np.array(out_init, dtype=np.uint16, copy=True)

@@ -1,0 +1,134 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the header declares, and rejects bad arguments with the documented status
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dit_token_b200 as dit
+from dit_token_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dit_token.h")
+
+OK, NULL, SHAPE, ALIGN, UNSUP = 0, 1, 2, 3, 4
+P = 0x10000  # an aligned, never dereferenced fake device address
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return dit.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DIT_API\s+[\w\s\*]+?\b(dit_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) == 8, names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.dit_abi_version() == 1
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.dit_status_string(s).decode().startswith(dit.STATUS[s])
+    assert L.dit_status_string(99) == b"unknown dit_status"
+
+
+def qk(L, **kw):
+    a = dict(q=P, qs=256, k=P, ks=256, wq=P, wk=P, cs=P, cp=P, B=1, rows=16, hq=2, hk=2, d=128,
+             grid=None, st=0, sh=0, sw=0, theta=10000.0, eps=1e-6)
+    a.update(kw)
+    return L.dit_qk_rmsnorm_rope(a["q"], a["qs"], a["k"], a["ks"], a["wq"], a["wk"], a["cs"], a["cp"], a["B"],
+                                 a["rows"], a["hq"], a["hk"], a["d"], a["grid"], a["st"], a["sh"], a["sw"],
+                                 a["theta"], a["eps"], None)
+
+
+def test_qk_argument_checks(L):
+    assert qk(L, q=None) == NULL
+    assert qk(L, wk=None) == NULL
+    assert qk(L, cs=None) == NULL
+    assert qk(L, d=96) == UNSUP
+    assert qk(L, d=0) == SHAPE
+    assert qk(L, qs=255) == SHAPE            # stride smaller than heads * head_dim
+    assert qk(L, qs=264, q=P + 2) == ALIGN   # pointer not 16-byte aligned
+    assert qk(L, qs=260) == ALIGN            # stride not a multiple of 8
+    assert qk(L, B=-1) == SHAPE
+    assert qk(L, rows=-5) == SHAPE
+    assert qk(L, rows=1 << 31) == SHAPE
+    assert qk(L, grid=P, st=44, sh=42, sw=40) == SHAPE   # sections do not sum to head_dim
+    assert qk(L, grid=P, st=43, sh=43, sw=42) == SHAPE   # odd section
+    assert qk(L, grid=P, st=-2, sh=66, sw=64) == SHAPE
+    assert qk(L, theta=0.0) == SHAPE
+    assert qk(L, eps=float("nan")) == SHAPE
+    assert qk(L, grid=P + 2, st=44, sh=42, sw=42) == ALIGN
+
+
+def test_empty_batches_launch_nothing(L):
+    # nothing to do -> DIT_OK even with NULL tensors, and no CUDA call is made
+    assert qk(L, B=0, q=None, k=None, cs=None, cp=None) == OK
+    assert qk(L, rows=0, q=None, k=None) == OK
+    assert qk(L, hq=0, hk=0) == OK
+    assert L.dit_swiglu(None, 8, None, 8, None, 8, None, None, 0, 0, 8, None) == OK
+    assert L.dit_gated_residual(None, 8, None, 8, None, 8, None, 8, P, P, 3, 0, 8, None) == OK
+    assert L.dit_adaln_modulate(None, 8, None, 8, None, None, 8, P, P, 0, 64, 8, 1e-6, None) == OK
+
+
+def test_adaln_argument_checks(L):
+    def call(**kw):
+        a = dict(x=P, xs=64, o=P, os=64, sh=P, sc=P, ms=64, B=1, rows=4, C=64, eps=1e-6)
+        a.update(kw)
+        return L.dit_adaln_modulate(a["x"], a["xs"], a["o"], a["os"], a["sh"], a["sc"], a["ms"], P, P,
+                                    a["B"], a["rows"], a["C"], a["eps"], None)
+    assert call(x=None) == NULL and call(sc=None) == NULL
+    assert call(C=0) == SHAPE and call(xs=56) == SHAPE and call(ms=-8) == SHAPE
+    assert call(C=60, xs=64, os=64) == ALIGN
+    assert call(ms=12) == ALIGN
+    assert call(o=P + 8) == ALIGN
+    assert call(C=16392, xs=16392, os=16392) == UNSUP
+    assert call(eps=-1.0) == SHAPE
+
+
+def test_residual_and_swiglu_argument_checks(L):
+    def res(**kw):
+        a = dict(x=P, xs=64, y=P, ys=64, g=P, gs=64, o=P, os=64, B=2, rows=4, C=64)
+        a.update(kw)
+        return L.dit_gated_residual(a["x"], a["xs"], a["y"], a["ys"], a["g"], a["gs"], a["o"], a["os"], P, P,
+                                    a["B"], a["rows"], a["C"], None)
+    assert res(y=None) == NULL and res(g=None) == NULL
+    assert res(ys=32) == SHAPE and res(gs=-8) == SHAPE and res(C=-8) == SHAPE
+    assert res(gs=4) == ALIGN and res(y=P + 4) == ALIGN and res(C=36, xs=64, ys=64, os=64) == ALIGN
+
+    def sw(**kw):
+        a = dict(a=P, as_=128, b=P, bs=128, o=P, os=64, B=1, rows=4, I=64)
+        a.update(kw)
+        return L.dit_swiglu(a["a"], a["as_"], a["b"], a["bs"], a["o"], a["os"], P, P, a["B"], a["rows"], a["I"],
+                            None)
+    assert sw(b=None) == NULL and sw(o=None) == NULL
+    assert sw(os=32) == SHAPE and sw(I=0) == SHAPE
+    assert sw(b=P + 64 * 2 + 2) == ALIGN and sw(as_=132) == ALIGN
+
+
+def test_validate_argument_checks(L):
+    flag = P
+    assert L.dit_validate_seqlens(None, P, 1, 4, flag, None) == NULL
+    assert L.dit_validate_seqlens(P, P, 1, 4, None, None) == NULL
+    assert L.dit_validate_seqlens(P, P, -1, 4, flag, None) == SHAPE
+    assert L.dit_validate_seqlens(P + 2, P, 1, 4, flag, None) == ALIGN
+
+
+def test_binding_rejects_cpu_tensors_before_the_library():
+    import torch
+    x = torch.zeros(4, 8, dtype=torch.bfloat16)
+    cs = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises((TypeError, ValueError)):
+        dit.dit_gated_residual(x, x, torch.zeros(1, 8, dtype=torch.bfloat16), cs, cs)
+    with pytest.raises(TypeError):
+        dit.dit_swiglu(x.float(), x.float(), cs, cs)

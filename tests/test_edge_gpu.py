@@ -1,0 +1,182 @@
+"""GPU edge cases, every valid row compared with the oracle: ragged shapes
+(rows not a multiple of a CTA, widths not a multiple of a warp step),
+zero-length and length-1 sequences, a sequence that fills its padded slot,
+GQA, head_dim 64 with 3D sections, unit grid axes, strided (fused QKV)
+buffers, in-place use, hundreds of sequences, every adaLN team/vector
+variant up to the largest supported hidden size, empty batches, and
+malformed device descriptors (skipped rows, nothing written out of bounds,
+flagged by dit_validate_seqlens)."""
+import numpy as np
+import pytest
+import torch
+
+import dit_token_b200 as dit
+from dit_token_b200 import workloads as W
+import _parity as P
+from _util import tbits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from dit_token_b200 import build
+    build.build()
+
+
+def ragged(head_dim=128, sections=(44, 42, 42), hq=3, hk=1, hidden=2056, inner=1032, seed=3):
+    lengths = (1, 0, 37, 136, 300, 64)
+    padded = (8, 8, 40, 136, 304, 64)
+    grids = ((1, 1, 1), (0, 0, 0), (2, 3, 5), (4, 1, 6), (3, 7, 1), (0, 0, 0))
+    return W.custom("ragged", lengths, padded, hidden=hidden, num_q_heads=hq, num_k_heads=hk,
+                    head_dim=head_dim, inner=inner, grids=grids, sections=sections, seed=seed)
+
+
+def all_ops_full(w, in_place=False):
+    rows = w.valid_rows()
+    keep = P.untouched_rows(w)
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp)
+    qo, ko = P.oracle_qk(w, inp, rows)
+    P.assert_close(P.gather_rows(q, rows), qo[rows], "q")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], "k")
+    P.assert_untouched(q, inp["q"], keep, "q")
+    P.assert_untouched(k, inp["k"], keep, "k")
+
+    inp = W.adaln_inputs(w)
+    out = P.gpu_adaln(w, inp, in_place=in_place)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_adaln(w, inp, rows)[rows], "adaln")
+    P.assert_untouched(out, inp["x"] if in_place else inp["out"], keep, "adaln")
+
+    inp = W.residual_inputs(w)
+    out = P.gpu_residual(w, inp, in_place=in_place)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_residual(w, inp, rows)[rows], "residual")
+    P.assert_untouched(out, inp["x"] if in_place else inp["out"], keep, "residual")
+
+    inp = W.swiglu_inputs(w)
+    out = P.gpu_swiglu(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, inp, rows)[rows], "swiglu")
+    P.assert_untouched(out, inp["out"], keep, "swiglu")
+
+
+@pytest.mark.parametrize("in_place", [False, True])
+def test_ragged_batch(in_place):
+    all_ops_full(ragged(), in_place=in_place)
+
+
+def test_head_dim_64_with_3d_sections_and_gqa():
+    all_ops_full(ragged(head_dim=64, sections=(24, 20, 20), hq=4, hk=2, hidden=264, inner=520))
+
+
+def test_1d_only_and_degenerate_sections():
+    w = W.custom("1d", (77, 3), (80, 8), hidden=512, num_q_heads=2, num_k_heads=2, head_dim=128, inner=256)
+    all_ops_full(w)
+    # a 1 x 1 x W grid whose only section is w reproduces the 1D rotation
+    w3 = W.custom("1d", (77, 3), (80, 8), hidden=512, num_q_heads=2, num_k_heads=2, head_dim=128, inner=256,
+                  grids=((1, 1, 77), (1, 1, 3)), sections=(0, 0, 128))
+    inp = W.qk_inputs(w)
+    a = P.gpu_qk(w, inp)
+    b = P.gpu_qk(w3, inp)
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+
+
+def test_many_sequences():
+    rng = np.random.default_rng(11)
+    lengths = rng.integers(0, 21, 300)
+    padded = [-(-int(L) // 8) * 8 + 8 * int(rng.integers(0, 2)) for L in lengths]
+    grids = [(int(L) // 4, 2, 2) if L >= 4 else (0, 0, 0) for L in lengths]
+    w = W.custom("many", lengths, padded, hidden=256, num_q_heads=2, num_k_heads=2, head_dim=64, inner=264,
+                 grids=grids, sections=(22, 22, 20))
+    all_ops_full(w)
+
+
+def test_fused_qkv_slices_and_wide_out_stride():
+    w = ragged()
+    inp = W.qk_inputs(w)
+    qw, kw = w.qk_width
+    # [rows, q | k | v] buffer: q and k are column slices with row stride qw + 2 kw
+    qkv = torch.cat([inp["q"], inp["k"], inp["k"]], dim=1).cuda()
+    cs, cp, grid = P.device_packing(w)
+    rv = W.rows_view(qkv)
+    dit.dit_qk_rmsnorm_rope(rv[:, :qw], rv[:, qw:qw + kw], inp["q_weight"].cuda(), inp["k_weight"].cuda(),
+                            cs, cp, num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
+                            rope_grid=grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps)
+    q, k = P.gpu_qk(w, inp)
+    assert torch.equal(qkv[:, :qw].contiguous().view(torch.int16), q.view(torch.int16))
+    assert torch.equal(qkv[:, qw:qw + kw].contiguous().view(torch.int16), k.view(torch.int16))
+    assert torch.equal(qkv[:, qw + kw:].cpu().view(torch.int16), inp["k"].view(torch.int16))  # v untouched
+    # adaLN into a wider output buffer (row stride 3 * hidden)
+    inp = W.adaln_inputs(w)
+    wide = W.sentinel_like((inp["x"].shape[0], 3 * w.hidden)).cuda()
+    mod = inp["mod"].cuda()
+    dit.dit_adaln_modulate(W.rows_view(inp["x"].cuda()), mod[:, 0], mod[:, 1], cs, cp,
+                           out=W.rows_view(wide)[:, w.hidden:2 * w.hidden], eps=w.eps)
+    ref = P.gpu_adaln(w, inp)
+    assert torch.equal(wide[:, w.hidden:2 * w.hidden].contiguous().view(torch.int16), ref.view(torch.int16))
+    assert torch.all(wide[:, :w.hidden].view(torch.int16) == W.SENTINEL)
+
+
+@pytest.mark.parametrize("hidden", [8, 256, 264, 2048, 2056, 3072, 4096, 5120, 8192, 16384])
+def test_adaln_every_team_shape(hidden):
+    w = W.custom("adaln", (13, 6), (16, 8), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=hidden)
+    rows = w.valid_rows()
+    inp = W.adaln_inputs(w)
+    out = P.gpu_adaln(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_adaln(w, inp, rows)[rows], f"adaln {hidden}")
+    P.assert_untouched(out, inp["out"], P.untouched_rows(w), "adaln")
+
+
+def test_swiglu_extreme_activations():
+    w = W.custom("sw", (5,), (8,), hidden=8, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64)
+    inp = W.swiglu_inputs(w)
+    vals = torch.tensor([0.0, -0.0, 1.0, -1.0, 20.0, -20.0, 88.0, -88.0, 100.0, -100.0, 1e-3, -1e-3,
+                         3.0e4, -3.0e4, 0.5, -0.5] * 4, dtype=torch.float32)
+    ab = W.rows_view(inp["ab"])
+    ab[:5, :64] = vals.to(torch.bfloat16)
+    rows = w.valid_rows()
+    out = P.gpu_swiglu(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, inp, rows)[rows], "swiglu extremes")
+
+
+def test_empty_batches():
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    cs = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = torch.zeros(1, 64, dtype=torch.bfloat16, device="cuda")
+    out = torch.full_like(x, 7.0)
+    dit.dit_gated_residual(x, x, g, cs, cs, out=out)          # num_seqs = 0
+    dit.dit_swiglu(x, x, cs, cs, out=out)
+    w = W.custom("zero", (0, 0), (4, 4), hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64)
+    inp = W.residual_inputs(w)
+    o = P.gpu_residual(w, inp)                               # all sequences empty
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+    assert torch.equal(o.cpu().view(torch.int16), inp["out"].view(torch.int16))
+
+
+def test_malformed_device_descriptors_are_skipped_and_flagged():
+    w = W.custom("bad", (10, 6), (8, 8), hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64)
+    # sequence 0 claims 10 valid rows in an 8-row slot; the second slot ends
+    # past the 16-row buffer (cu_seqlens_padded = [0, 8, 20]).
+    inp = W.residual_inputs(w)
+    x, y, out = inp["x"].cuda(), inp["y"].cuda(), inp["out"].cuda()
+    mod = inp["mod"].cuda()
+    cs = torch.tensor([0, 10, 16], dtype=torch.int32, device="cuda")
+    cp = torch.tensor([0, 8, 20], dtype=torch.int32, device="cuda")
+    dit.dit_gated_residual(W.rows_view(x), W.rows_view(y), mod[:, 2], cs, cp, out=W.rows_view(out))
+    flag = dit.dit_validate_seqlens(cs, cp, 16)
+    torch.cuda.synchronize()
+    assert flag.tolist() == [1, 0]
+    o = out.cpu()
+    assert torch.all(o[:W.CANARY_ROWS].view(torch.int16) == W.SENTINEL)
+    assert torch.all(o[-W.CANARY_ROWS:].view(torch.int16) == W.SENTINEL)
+    # rows 0..7 (sequence 0, clamped to its slot) and 8..13 (sequence 1) are written
+    assert not torch.any(o[W.CANARY_ROWS:W.CANARY_ROWS + 14].view(torch.int16) == W.SENTINEL)
+    assert torch.all(o[W.CANARY_ROWS + 14:W.CANARY_ROWS + 16].view(torch.int16) == W.SENTINEL)
+    good = dit.dit_validate_seqlens(torch.tensor([0, 6, 12], dtype=torch.int32, device="cuda"),
+                                    torch.tensor([0, 8, 16], dtype=torch.int32, device="cuda"), 16)
+    cp2 = torch.tensor([0, 8, 16], dtype=torch.int32, device="cuda")
+    cs2 = torch.tensor([0, 5, 4], dtype=torch.int32, device="cuda")   # decreasing
+    bad2 = dit.dit_validate_seqlens(cs2, cp2, 16)
+    torch.cuda.synchronize()
+    assert good.tolist()[0] == 0 and bad2.tolist() == [1, 1]
