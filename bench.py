@@ -213,37 +213,62 @@ class Step:
         self.rx, self.ry, self.rout = dev(host["res"]["x"]), dev(host["res"]["y"]), dev(host["res"]["out"])
         self.ab, self.sout = dev(host["swiglu"]["ab"]), dev(host["swiglu"]["out"])
 
-    def inputs(self):
-        """(device tensor, name) of every input the step consumes."""
-        return [(self.q, "q"), (self.k, "k"), (self.ax, "adaln_x"), (self.rx, "res_x"), (self.ry, "res_y"),
-                (self.ab, "ab")]
+    def op_inputs(self, op):
+        """Device tensors an op reads (what a host-resident caller must upload)."""
+        return {"qk_rmsnorm_rope": [self.q, self.k], "adaln_modulate": [self.ax],
+                "gated_residual": [self.rx, self.ry], "swiglu": [self.ab]}[op]
 
-    def outputs(self):
-        return [(self.q, "q"), (self.k, "k"), (self.aout, "adaln_out"), (self.rout, "res_out"),
-                (self.sout, "swiglu_out")]
+    def op_outputs(self, op):
+        """Device tensors an op writes (what the caller reads back)."""
+        return {"qk_rmsnorm_rope": [self.q, self.k], "adaln_modulate": [self.aout],
+                "gated_residual": [self.rout], "swiglu": [self.sout]}[op]
+
+    def run_op(self, op):
+        w, d, rv = self.w, self.dit, W.rows_view
+        if op == "qk_rmsnorm_rope":
+            d.dit_qk_rmsnorm_rope(rv(self.q), rv(self.k), self.wq, self.wk, self.cs, self.cp,
+                                  num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
+                                  rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps)
+        elif op == "adaln_modulate":
+            d.dit_adaln_modulate(rv(self.ax), self.mod[:, 0], self.mod[:, 1], self.cs, self.cp,
+                                 out=rv(self.aout), eps=w.eps)
+        elif op == "gated_residual":
+            d.dit_gated_residual(rv(self.rx), rv(self.ry), self.mod[:, 2], self.cs, self.cp, out=rv(self.rout))
+        else:
+            ab = rv(self.ab)
+            d.dit_swiglu(ab[:, : w.inner], ab[:, w.inner:], self.cs, self.cp, out=rv(self.sout))
 
     def run(self, events=None):
-        w, d, rv = self.w, self.dit, W.rows_view
-        ev = events or {}
-        def mark(op, i):
-            if op in ev:
-                ev[op][i].record()
-        mark("qk_rmsnorm_rope", 0)
-        d.dit_qk_rmsnorm_rope(rv(self.q), rv(self.k), self.wq, self.wk, self.cs, self.cp,
-                              num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
-                              rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps)
-        mark("qk_rmsnorm_rope", 1)
-        mark("adaln_modulate", 0)
-        d.dit_adaln_modulate(rv(self.ax), self.mod[:, 0], self.mod[:, 1], self.cs, self.cp, out=rv(self.aout),
-                             eps=w.eps)
-        mark("adaln_modulate", 1)
-        mark("gated_residual", 0)
-        d.dit_gated_residual(rv(self.rx), rv(self.ry), self.mod[:, 2], self.cs, self.cp, out=rv(self.rout))
-        mark("gated_residual", 1)
-        mark("swiglu", 0)
-        ab = rv(self.ab)
-        d.dit_swiglu(ab[:, : w.inner], ab[:, w.inner:], self.cs, self.cp, out=rv(self.sout))
-        mark("swiglu", 1)
+        for op in OPS:
+            if events:
+                events[op][0].record()
+            self.run_op(op)
+            if events:
+                events[op][1].record()
+
+
+def time_next_ops(step: Step, steps: int, warmup: int, device) -> dict:
+    """Mean launch time of the operators built beyond the four-op step (same
+    buffers, same stream), each timed on its own."""
+    w, d, rv = step.w, step.dit, W.rows_view
+
+    def fused():
+        d.dit_gated_residual_adaln(rv(step.rx), rv(step.ry), step.mod[:, 2], step.mod[:, 3], step.mod[:, 4],
+                                   step.cs, step.cp, res_out=rv(step.rout), norm_out=rv(step.aout), eps=w.eps)
+
+    out = {}
+    for name, fn in (("gated_residual_adaln", fused),):
+        for _ in range(warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(device)
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(device)
+        out[name] = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    return out
 
 
 def host_inputs(w: W.Workload) -> dict:
@@ -276,33 +301,63 @@ def time_device(step: Step, steps: int, warmup: int, device):
     return elapsed_ms, op_ms, (t_host0, t_host1)
 
 
-def time_e2e(step: Step, steps: int, warmup: int, device):
-    """Same step through the public API, inputs copied from pinned host memory
-    and results copied back to pinned host memory inside the timed region."""
-    stream = torch.cuda.current_stream(device)
-    h_in = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t, _ in step.inputs()]
-    h_out = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t, _ in step.outputs()]
-    for d, h in h_in:
-        h.copy_(d)
-    h2d = sum(h.numel() * h.element_size() for _, h in h_in)
-    d2h = sum(h.numel() * h.element_size() for _, h in h_out)
+def time_e2e(sets, steps: int, warmup: int, device):
+    """The same step through the public API for a caller whose data lives in
+    pinned host memory: every step uploads each op's inputs, runs the op and
+    downloads its outputs, all inside the timed region.  Uploads, kernels and
+    downloads run on three streams ordered by events, so the two copy
+    directions overlap each other and the kernels; two device buffer sets
+    alternate between steps (q and k are updated in place)."""
+    h_in = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_inputs(op)]
+            for op in OPS}
+    h_out = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_outputs(op)]
+             for op in OPS}
+    for op in OPS:
+        for h, d in zip(h_in[op], sets[0].op_inputs(op)):
+            h.copy_(d)
+    h2d = sum(h.numel() * h.element_size() for op in OPS for h in h_in[op])
+    d2h = sum(h.numel() * h.element_size() for op in OPS for h in h_out[op])
+    s_up, s_run, s_down = (torch.cuda.Stream(device) for _ in range(3))
+    free = [None, None]
 
-    def one():
-        for d, h in h_in:
-            d.copy_(h, non_blocking=True)
-        step.run()
-        for d, h in h_out:
-            h.copy_(d, non_blocking=True)
+    def one(k):
+        st = sets[k % 2]
+        ready, done = {}, {}
+        with torch.cuda.stream(s_up):
+            if free[k % 2] is not None:
+                s_up.wait_event(free[k % 2])
+            for op in OPS:
+                for d, h in zip(st.op_inputs(op), h_in[op]):
+                    d.copy_(h, non_blocking=True)
+                ready[op] = torch.cuda.Event()
+                ready[op].record(s_up)
+        with torch.cuda.stream(s_run):
+            for op in OPS:
+                s_run.wait_event(ready[op])
+                st.run_op(op)
+                done[op] = torch.cuda.Event()
+                done[op].record(s_run)
+        with torch.cuda.stream(s_down):
+            for op in OPS:
+                s_down.wait_event(done[op])
+                for h, d in zip(h_out[op], st.op_outputs(op)):
+                    h.copy_(d, non_blocking=True)
+            free[k % 2] = torch.cuda.Event()
+            free[k % 2].record(s_down)
 
-    for _ in range(warmup):
-        one()
+    for k in range(warmup):
+        one(k)
     barrier()
     torch.cuda.synchronize(device)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        one()
-    end.record(stream)
+    start.record(s_up)
+    s_run.wait_stream(s_up)
+    s_down.wait_stream(s_up)
+    for k in range(steps):
+        one(k)
+    s_down.wait_stream(s_run)
+    s_down.wait_stream(s_up)
+    end.record(s_down)
     torch.cuda.synchronize(device)
     barrier()
     return start.elapsed_time(end), h2d, d2h
@@ -400,7 +455,7 @@ def run_dit(args):
     if rank == 0 or world == 1:
         build.build()
     barrier()
-    w0 = W.workload(args.workload, args.seed)
+    w0 = W.scaled(W.workload(args.workload, args.seed), args.scale)
     w = dataclasses.replace(w0, seed=data_seed(args.seed, rank))
     host = host_inputs(w)
     step = Step(w, host, device)
@@ -411,8 +466,9 @@ def run_dit(args):
     clocks = sampler.summary(h0, h1)
     max_ms = reduce_max(elapsed_ms, device)
     op_ms_max = {op: reduce_max(v, device) for op, v in op_ms.items()}
+    next_ms = {k: reduce_max(v, device) for k, v in time_next_ops(step, args.steps, args.warmup, device).items()}
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    e2e_ms, h2d, d2h = time_e2e(step, e2e_steps, min(args.warmup, 3), device)
+    e2e_ms, h2d, d2h = time_e2e([step, Step(w, host, device)], e2e_steps, min(args.warmup, 3), device)
     e2e_max = reduce_max(e2e_ms, device)
 
     tokens = w.num_valid * world
@@ -440,8 +496,17 @@ def run_dit(args):
                      "frac": round(dom_gbs / peak, 4), "traffic": profiled_traffic(dom, w.name),
                      "algorithmic_bytes": abytes[dom]},
         "gpu_launches": len(OPS) * args.steps,
+        "next_ops": {
+            "gated_residual_adaln": {
+                "us": round(next_ms["gated_residual_adaln"] * 1e3, 2),
+                "gbs": round(8 * w.hidden * w.num_valid / (next_ms["gated_residual_adaln"] / 1e3) / 1e9, 1),
+                "bytes": 8 * w.hidden * w.num_valid,
+                "unfused_us": round((op_ms_max["gated_residual"] + op_ms_max["adaln_modulate"]) * 1e3, 2)},
+        },
         "e2e": {"value": round(tokens * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": round(e2e_max / e2e_steps, 3),
+                "schedule": "per-op upload / kernel / download on 3 streams, 2 device buffer sets"},
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -456,7 +521,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return  # the CPU oracle runs once, on rank 0
-    w = W.workload(args.workload, args.seed)
+    w = W.scaled(W.workload(args.workload, args.seed), args.scale)
     host = host_inputs(w)
     runner = OracleRunner(w, host)
     per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
@@ -489,6 +554,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("dit", "reference"), default="dit")
     ap.add_argument("--workload", default="batched_varlen", choices=W.WORKLOAD_NAMES)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="scale every sequence's valid length (a smaller batch of the same shapes, "
+                         "e.g. for profiling); the JSON names the scaled workload")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

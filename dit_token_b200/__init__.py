@@ -13,6 +13,8 @@ The operators (see the header for the exact definitions):
 * ``dit_adaln_modulate``   LN(x) * (1 + scale_b) + shift_b
 * ``dit_gated_residual``   x + gate_b * y
 * ``dit_swiglu``           silu(a) * b
+* ``dit_gated_residual_adaln``  res = x + gate_b * y, then LN(res) * (1 + scale_b) + shift_b
+* ``dit_frames_to_u8``     decoded fp32 frames [B, C, T, H, W] -> uint8 BTHWC (or planar BTCHW)
 
 All run over a packed sequence described by ``cu_seqlens`` (cumulative valid
 lengths) and ``cu_seqlens_padded`` (row offsets), touching valid rows only.
@@ -26,9 +28,12 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = ["dit_qk_rmsnorm_rope", "dit_adaln_modulate", "dit_gated_residual", "dit_swiglu",
+           "dit_gated_residual_adaln", "dit_frames_to_u8",
            "dit_validate_seqlens", "DitError", "library", "LIB_PATH", "STATUS"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_token.so")
+# DIT_TOKEN_LIB may point at another build of the same library.
+LIB_PATH = os.environ.get("DIT_TOKEN_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                          "libdit_token.so")
 
 STATUS = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_ALIGN",
           4: "DIT_ERR_UNSUPPORTED", 5: "DIT_ERR_SEQLENS", 6: "DIT_ERR_CUDA"}
@@ -53,7 +58,10 @@ _SIGNATURES = {
     "dit_adaln_modulate": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _VP],
     "dit_gated_residual": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
     "dit_swiglu": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
+    "dit_gated_residual_adaln": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _I64, _VP, _I64,
+                                 _VP, _VP, _I32, _I64, _I32, _F32, _VP],
     "dit_validate_seqlens": [_VP, _VP, _I32, _I64, _VP, _VP],
+    "dit_frames_to_u8": [_VP, _I64, _I64, _I64, _I64, _I64, _I32, _VP, _VP],
     "dit_status_string": [_I32],
     "dit_last_cuda_error": [],
     "dit_abi_version": [],
@@ -205,6 +213,32 @@ def dit_gated_residual(x: torch.Tensor, y: torch.Tensor, gate: torch.Tensor,
     return out
 
 
+def dit_gated_residual_adaln(x: torch.Tensor, y: torch.Tensor, gate: torch.Tensor, shift: torch.Tensor,
+                             scale: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, *,
+                             res_out: Optional[torch.Tensor] = None, norm_out: Optional[torch.Tensor] = None,
+                             eps: float = 1e-6, stream=None):
+    """res = x + gate_b * y; norm = LayerNorm(res) * (1 + scale_b) + shift_b,
+    on valid rows, in one pass.  ``res_out`` may be x.  Returns (res, norm)."""
+    hidden = x.size(-1)
+    if res_out is None:
+        res_out = torch.empty_like(x)
+    if norm_out is None:
+        norm_out = torch.empty_like(x)
+    xp, xs = _rows(x, "x")
+    yp, ys = _rows(y, "y")
+    rp, rs = _rows(res_out, "res_out")
+    np_, ns = _rows(norm_out, "norm_out")
+    gp, gst = _seq_vectors(gate, hidden, "gate")
+    shp, sst = _seq_vectors(shift, hidden, "shift")
+    scp, cst = _seq_vectors(scale, hidden, "scale")
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    if B > 1 and sst != cst:
+        raise ValueError("shift and scale must share one sequence stride")
+    _call("dit_gated_residual_adaln", xp, xs, yp, ys, gp, gst if B > 1 else hidden, shp, scp,
+          sst if B > 1 else hidden, rp, rs, np_, ns, cs, cp, B, x.size(0), hidden, float(eps), _stream(stream))
+    return res_out, norm_out
+
+
 def dit_swiglu(a: torch.Tensor, b: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor,
                *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """out = silu(a) * b on valid rows.  a, b: [rows, inner] (e.g. the two
@@ -219,6 +253,23 @@ def dit_swiglu(a: torch.Tensor, b: torch.Tensor, cu_seqlens: torch.Tensor, cu_se
     op, os_ = _rows(out, "out")
     cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
     _call("dit_swiglu", ap, as_, bp, bs, op, os_, cs, cp, B, a.size(0), inner, _stream(stream))
+    return out
+
+
+def dit_frames_to_u8(x: torch.Tensor, *, layout: str = "bthwc", out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Decoded frames fp32 [B, C, T, H, W] -> uint8 [B, T, H, W, C] ("bthwc") or
+    [B, T, C, H, W] ("btchw"): u = rint(clamp((x + 1) * 127.5, 0, 255))."""
+    if x.dtype != torch.float32 or not x.is_cuda or x.dim() != 5 or not x.is_contiguous():
+        raise TypeError("x: expected a contiguous float32 CUDA tensor [B, C, T, H, W]")
+    B, C, T, H, Wd = x.shape
+    code = {"bthwc": 0, "btchw": 1}[layout]
+    shape = (B, T, H, Wd, C) if code == 0 else (B, T, C, H, Wd)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    if out.dtype != torch.uint8 or not out.is_cuda or tuple(out.shape) != shape or not out.is_contiguous():
+        raise TypeError(f"out: expected a contiguous uint8 CUDA tensor {shape}")
+    _call("dit_frames_to_u8", x.data_ptr(), B, C, T, H, Wd, code, out.data_ptr(), _stream(stream))
     return out
 
 

@@ -174,6 +174,42 @@ dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const void* y
     return from_cuda(dit::launch_gated_residual(p, static_cast<cudaStream_t>(stream)));
 }
 
+dit_status dit_gated_residual_adaln(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                                    const void* gate, int64_t gate_seq_stride,
+                                    const void* shift, const void* scale, int64_t mod_seq_stride,
+                                    void* res_out, int64_t res_row_stride, void* norm_out, int64_t norm_row_stride,
+                                    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
+                                    void* stream)
+{
+    bool empty = false;
+    dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
+    if (st != DIT_OK)
+        return st;
+    if (hidden <= 0 || x_row_stride < hidden || y_row_stride < hidden || res_row_stride < hidden ||
+        norm_row_stride < hidden || gate_seq_stride < 0 || mod_seq_stride < 0 || !(eps >= 0.f) ||
+        !std::isfinite(eps))
+        return DIT_ERR_SHAPE;
+    if (hidden > dit::kMaxAdalnHidden)
+        return DIT_ERR_UNSUPPORTED;
+    if (empty)
+        return DIT_OK;
+    if (!x || !y || !gate || !shift || !scale || !res_out || !norm_out)
+        return DIT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(gate) || !aligned16(shift) || !aligned16(scale) ||
+        !aligned16(res_out) || !aligned16(norm_out) || !mult8(hidden) || !mult8(x_row_stride) ||
+        !mult8(y_row_stride) || !mult8(res_row_stride) || !mult8(norm_row_stride) || !mult8(gate_seq_stride) ||
+        !mult8(mod_seq_stride))
+        return DIT_ERR_ALIGN;
+    dit::FusedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y),
+                       static_cast<const uint16_t*>(gate), static_cast<const uint16_t*>(shift),
+                       static_cast<const uint16_t*>(scale), static_cast<uint16_t*>(res_out),
+                       static_cast<uint16_t*>(norm_out), x_row_stride, y_row_stride, gate_seq_stride,
+                       mod_seq_stride, res_row_stride, norm_row_stride,
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps};
+    return from_cuda(dit::launch_gated_residual_adaln(p, static_cast<cudaStream_t>(stream)));
+}
+
 dit_status dit_swiglu(const void* a, int64_t a_row_stride, const void* b, int64_t b_row_stride,
                       void* out, int64_t out_row_stride,
                       const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
@@ -196,6 +232,26 @@ dit_status dit_swiglu(const void* a, int64_t a_row_stride, const void* b, int64_
                         static_cast<uint16_t*>(out), a_row_stride, b_row_stride, out_row_stride,
                         packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), inner};
     return from_cuda(dit::launch_swiglu(p, static_cast<cudaStream_t>(stream)));
+}
+
+dit_status dit_frames_to_u8(const float* x, int64_t batch, int64_t channels, int64_t frames, int64_t height,
+                            int64_t width, int32_t layout, uint8_t* out, void* stream)
+{
+    if (batch < 0 || channels < 0 || frames < 0 || height < 0 || width < 0)
+        return DIT_ERR_SHAPE;
+    if (layout != DIT_FRAMES_BTHWC && layout != DIT_FRAMES_BTCHW)
+        return DIT_ERR_UNSUPPORTED;
+    if (batch == 0 || channels == 0 || frames == 0 || height == 0 || width == 0)
+        return DIT_OK;
+    const double total = (double)batch * channels * frames * height * width;
+    if (total > 9.0e15)
+        return DIT_ERR_SHAPE;
+    if (!x || !out)
+        return DIT_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) & 3u)
+        return DIT_ERR_ALIGN;
+    dit::FramesParams p{x, out, batch, channels, frames, height, width, layout};
+    return from_cuda(dit::launch_frames_to_u8(p, static_cast<cudaStream_t>(stream)));
 }
 
 dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,

@@ -95,6 +95,22 @@ __device__ __forceinline__ uint4 ld_shared_vec(const uint16_t* p)
     return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// Asynchronous 16-byte global -> shared copies (L1 bypassed), completed with
+// commit/wait groups: a hardware wait, no polling loop.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------ bf16 <-> fp32
 // A bf16 value is the upper half of a binary32 value, so widening is a shift.
 
@@ -109,6 +125,21 @@ __device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
     f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
 }
 
+// The same widening as an opaque instruction, so that a later pass over
+// register-resident packed data recomputes it instead of keeping eight fp32
+// copies per vector alive (which would cost occupancy in the row kernels).
+__device__ __forceinline__ void unpack8_again(uint4 v, float (&f)[8])
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t lo, hi;
+        asm volatile("shl.b32 %0, %2, 16;\n\tand.b32 %1, %2, 0xffff0000;" : "=r"(lo), "=r"(hi) : "r"(w[i]));
+        f[2 * i] = __uint_as_float(lo);
+        f[2 * i + 1] = __uint_as_float(hi);
+    }
+}
+
 // Two fp32 values -> one bf16x2 word (round to nearest, ties to even).
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
@@ -121,6 +152,28 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8])
 {
     return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
+
+// Barrier among the TEAM warps of team `team` only (hardware named barrier
+// 1 + team; id 0 stays __syncthreads'), so the row teams of one CTA never
+// wait for each other.
+template <int TEAM>
+__device__ __forceinline__ void team_barrier(int team)
+{
+    if (TEAM == kWarpsPerCta)
+        __syncthreads();
+    else
+        asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "n"(TEAM * kWarp) : "memory");
+}
+
+// Minimum resident CTAs per SM to ask of a row kernel holding VPT 16-byte
+// vectors per lane of each of INPUTS streamed inputs at once (about
+// 4 * INPUTS * VPT + 28 registers per thread).
+template <int VPT, int INPUTS = 1>
+struct MinCtas {
+    static constexpr int regs = 4 * INPUTS * VPT + 28;
+    static constexpr int raw = 65536 / (kCtaThreads * regs);
+    static constexpr int value = raw < 1 ? 1 : (raw > 8 ? 8 : raw);
+};
 
 template <int WIDTH>
 __device__ __forceinline__ float group_sum(float v)

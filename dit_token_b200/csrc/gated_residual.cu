@@ -14,7 +14,10 @@
 namespace dit {
 namespace {
 
-constexpr int kUnroll = 4;
+#ifndef DIT_EW_UNROLL
+#define DIT_EW_UNROLL 4
+#endif
+constexpr int kUnroll = DIT_EW_UNROLL;  // 16-byte vectors per lane and input in flight
 
 __global__ void __launch_bounds__(kCtaThreads)
 gated_residual_kernel(const GatedParams p)

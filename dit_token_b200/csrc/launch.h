@@ -63,6 +63,25 @@ struct GatedParams {
     int32_t hidden;
 };
 
+struct FusedParams {
+    const uint16_t* x;
+    const uint16_t* y;
+    const uint16_t* gate;
+    const uint16_t* shift;
+    const uint16_t* scale;
+    uint16_t* res_out;
+    uint16_t* norm_out;
+    int64_t x_row_stride;
+    int64_t y_row_stride;
+    int64_t gate_seq_stride;
+    int64_t mod_seq_stride;
+    int64_t res_row_stride;
+    int64_t norm_row_stride;
+    Packing pk;
+    int32_t hidden;
+    float eps;
+};
+
 struct SwigluParams {
     const uint16_t* a;
     const uint16_t* b;
@@ -74,10 +93,19 @@ struct SwigluParams {
     int32_t inner;
 };
 
+struct FramesParams {
+    const float* x;
+    uint8_t* out;
+    int64_t B, C, T, H, W;
+    int32_t layout;
+};
+
+cudaError_t launch_frames_to_u8(const FramesParams& p, cudaStream_t stream);
 cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_adaln_modulate(const AdalnParams& p, cudaStream_t stream);
 cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream);
 cudaError_t launch_swiglu(const SwigluParams& p, cudaStream_t stream);
+cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream);
 cudaError_t launch_validate_seqlens(const Packing& pk, int64_t num_rows_padded, int32_t* flag,
                                     cudaStream_t stream);
 

@@ -21,7 +21,10 @@
 namespace dit {
 namespace {
 
-constexpr int kUnroll = 4;
+#ifndef DIT_QK_UNROLL
+#define DIT_QK_UNROLL 4
+#endif
+constexpr int kUnroll = DIT_QK_UNROLL;  // head vectors per lane in flight
 
 // angle mod 2*pi in fp64, then single precision: keeps the angle exact to
 // ~1e-7 rad for any position, and lets sincosf take its short path.

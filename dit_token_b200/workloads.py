@@ -140,6 +140,28 @@ def workload(name: str, seed: int = 0) -> Workload:
     raise KeyError(f"unknown workload {name!r}; known: {WORKLOAD_NAMES}")
 
 
+def scaled(w: Workload, factor: float) -> Workload:
+    """The same workload with every sequence's valid length scaled by
+    ``factor`` (a smaller or larger batch of the same shapes): padding keeps
+    the workload's granularity and video grids keep their 24 x 42 frames."""
+    if factor == 1.0:
+        return w
+    gran = {"tiny": 256, "single_stream": 128, "video": 256, "long_video": 256, "batched_varlen": 128}
+    g = gran.get(w.name.split("@")[0], 8)
+    lengths = tuple(max(1, int(round(L * factor))) for L in w.lengths)
+    padded = tuple(_round_up(L, g) for L in lengths)
+    grids = None
+    if w.grids is not None:
+        frame = _FRAME_H * _FRAME_W
+        if w.name.startswith("batched_varlen"):
+            grids = tuple((L // frame, _FRAME_H, _FRAME_W) for L in lengths)
+        else:  # keep the audio tail, shrink the frames
+            grids = tuple((max(0, (L - (L0 - T * H * Wd)) // frame), _FRAME_H, _FRAME_W)
+                          for L, L0, (T, H, Wd) in zip(lengths, w.lengths, w.grids))
+    return Workload(f"{w.name}@{factor:g}", lengths, padded, w.hidden, w.num_q_heads, w.num_k_heads,
+                    w.head_dim, w.inner, grids, w.sections, w.rope_theta, w.eps, w.seed)
+
+
 def custom(name: str, lengths, padded, *, hidden, num_q_heads, num_k_heads, head_dim, inner,
            grids=None, sections=(0, 0, 0), rope_theta=10000.0, eps=1e-6, seed=0) -> Workload:
     """A workload with explicit shapes (edge cases, small ragged tests)."""
@@ -247,6 +269,31 @@ def swiglu_inputs(w: Workload) -> dict:
     """A chunked [rows, 2 * inner] buffer: a = columns [0, inner), b = the rest."""
     ab = _row_buffer(w, 2 * w.inner, "ab")
     return {"ab": ab, "a": ab[:, : w.inner], "b": ab[:, w.inner:], "out": _row_buffer(w, w.inner, None)}
+
+
+# Decoded-video frames of the pages' 10-second request: 243 frames of
+# 1344 x 768 RGB ("MiniMax H3 通过 vLLM-Omni 实现 FastH3 实时推理", results and
+# duration-sweep tables), in the decoder's channels-first layout.
+FRAMES_SHAPE = (1, 3, 243, 768, 1344)
+
+
+def frames_input(shape=FRAMES_SHAPE, seed: int = 0) -> torch.Tensor:
+    """fp32 [B, C, T, H, W] decoder output: uniform in [-1.05, 1.05] (slightly
+    past the nominal [-1, 1] so the clamps are exercised), seeded, chunked
+    like the normal draws."""
+    n = int(math.prod(shape))
+    out = torch.empty(n, dtype=torch.float32)
+    nchunks = max(1, -(-n // _CHUNK))
+    children = np.random.SeedSequence(seed).spawn(nchunks)
+
+    def fill(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        g = np.random.Generator(np.random.PCG64(children[i]))
+        out[lo:hi] = torch.from_numpy(g.uniform(-1.05, 1.05, hi - lo).astype(np.float32))
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(fill, range(nchunks)))
+    return out.view(*shape)
 
 
 def sample_rows(w: Workload, per_seq: int, seed: int = 1234) -> np.ndarray:

@@ -134,6 +134,30 @@ DIT_API dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const
                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
                               int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, void* stream);
 
+/* Gated residual update fused with the next sublayer's adaLN modulation:
+ *   res_out  = bf16(x + gate_b * y)
+ *   norm_out = bf16(LN(res_out) * (1 + scale_b) + shift_b)
+ * LN (no affine, biased variance) reads the residual as stored in bf16, so the
+ * pair equals dit_gated_residual followed by dit_adaln_modulate on its output,
+ * while x and y are read once and res_out and norm_out written once.
+ *
+ * Pages: first page "Key takeaways" bullet 2 (residual updates fused together
+ * with the modulation and normalization work).
+ * x, y         device bf16 [num_rows_padded][hidden] with their own row strides
+ * gate         device bf16, vector of sequence b at gate + b * gate_seq_stride
+ * shift, scale device bf16, vectors of sequence b at + b * mod_seq_stride
+ * res_out      device bf16 [num_rows_padded][hidden] (may be x)
+ * norm_out     device bf16 [num_rows_padded][hidden] (must not overlap the others)
+ * hidden       a multiple of 8, at most 16384
+ */
+DIT_API dit_status dit_gated_residual_adaln(const void* x, int64_t x_row_stride, const void* y,
+                                            int64_t y_row_stride, const void* gate, int64_t gate_seq_stride,
+                                            const void* shift, const void* scale, int64_t mod_seq_stride,
+                                            void* res_out, int64_t res_row_stride, void* norm_out,
+                                            int64_t norm_row_stride, const int32_t* cu_seqlens,
+                                            const int32_t* cu_seqlens_padded, int32_t num_seqs,
+                                            int64_t num_rows_padded, int32_t hidden, float eps, void* stream);
+
 /* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)).
  *
  * Pages: first page "Key takeaways" bullet 2 and third page "vLLM-Omni 中的
@@ -147,6 +171,28 @@ DIT_API dit_status dit_swiglu(const void* a, int64_t a_row_stride, const void* b
                       void* out, int64_t out_row_stride,
                       const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
                       int32_t num_seqs, int64_t num_rows_padded, int32_t inner, void* stream);
+
+/* Decoded video frames (fp32) -> uint8, converted once on the device before
+ * the media encoder.
+ *
+ * Pages: first page "Key takeaways" bullet 3 (frames are converted on the GPU
+ * to compact uint8 BTHWC data, and the encoder reads planar paths); third
+ * page "vLLM-Omni 中的系统级优化" bullet 4 (the FP32 frames are converted to
+ * contiguous uint8 only once).  The pages give no value mapping; each value
+ * becomes u = rint(clamp((x + 1) * 127.5, 0, 255)) computed in fp32 (x + 1
+ * rounded, then * 127.5 rounded), ties to even, NaN -> 0.
+ *
+ * x       device fp32 [batch][channels][frames][height][width], contiguous, 4-byte aligned
+ * layout  DIT_FRAMES_BTHWC: out [batch][frames][height][width][channels] (interleaved)
+ *         DIT_FRAMES_BTCHW: out [batch][frames][channels][height][width] (planes)
+ * out     device uint8, batch*channels*frames*height*width bytes, contiguous
+ * Fast path when width % 16 == 0, channels is 1, 3 or 4 and both pointers are
+ * 16-byte aligned; any other shape takes a per-value path with the same result.
+ */
+#define DIT_FRAMES_BTHWC 0
+#define DIT_FRAMES_BTCHW 1
+DIT_API dit_status dit_frames_to_u8(const float* x, int64_t batch, int64_t channels, int64_t frames,
+                                    int64_t height, int64_t width, int32_t layout, uint8_t* out, void* stream);
 
 /* Device-side check of a packing descriptor; no counterpart on the pages (it
  * guards the padding-free packing of the first page, "Key takeaways" bullet 1).

@@ -43,10 +43,16 @@ def lib() -> ctypes.CDLL:
             u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
         L.oracle_gated_residual.argtypes = [
             u16p, i64, u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
+        L.oracle_gated_residual_adaln.argtypes = [
+            u16p, i64, u16p, i64, u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64,
+            u16p, i64, u16p, i64, f64p, i64p, i64]
         L.oracle_swiglu.argtypes = [
             u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
-        for name in ("oracle_qk_rmsnorm_rope", "oracle_adaln_modulate",
-                     "oracle_gated_residual", "oracle_swiglu", "oracle_num_threads"):
+        L.oracle_frames_to_u8.argtypes = [ctypes.POINTER(ctypes.c_float), i64, i64, i64, i64, i64, i32,
+                                          ctypes.POINTER(ctypes.c_uint8)]
+        for name in ("oracle_qk_rmsnorm_rope", "oracle_adaln_modulate", "oracle_frames_to_u8",
+                     "oracle_gated_residual", "oracle_gated_residual_adaln", "oracle_swiglu",
+                     "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -205,6 +211,38 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
     return (out, o64) if want_f64 else out
 
 
+def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
+                        gate_seq_stride=None, mod_seq_stride=None, x_row_stride=None, y_row_stride=None,
+                        rows=None, res_init=None, norm_init=None, want_f64=False, res_out=None,
+                        norm_out=None):
+    """res = x + gate_b * y (bf16), norm = LN(res) * (1 + scale_b) + shift_b on
+    valid rows.  Returns (res, norm) or, with want_f64, (res, norm, norm_f64)."""
+    cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
+    B = cs.size - 1
+    x, xs = _flat_view(x, x_row_stride, None)
+    y, ys = _flat_view(y, y_row_stride, None)
+    nrows = x.shape[0]
+    if res_out is None:
+        res_out = np.array(x if res_init is None else res_init, dtype=np.uint16, copy=True)
+    if norm_out is None:
+        norm_out = np.array(x if norm_init is None else norm_init, dtype=np.uint16, copy=True)
+    n64 = np.full(norm_out.shape, np.nan) if want_f64 else None
+    g = np.ascontiguousarray(_u16(gate))
+    sh = np.ascontiguousarray(_u16(shift))
+    sc = np.ascontiguousarray(_u16(scale))
+    gss = hidden if gate_seq_stride is None else gate_seq_stride
+    mss = hidden if mod_seq_stride is None else mod_seq_stride
+    r, nr = _rows(rows)
+    rc = lib().oracle_gated_residual_adaln(
+        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _ptr(g, ctypes.c_uint16), gss,
+        _ptr(sh, ctypes.c_uint16), _ptr(sc, ctypes.c_uint16), mss,
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
+        _ptr(res_out, ctypes.c_uint16), xs, _ptr(norm_out, ctypes.c_uint16), xs, _ptr(n64, ctypes.c_double),
+        _ptr(r, ctypes.c_int64), nr)
+    _check(rc, "gated_residual_adaln")
+    return (res_out, norm_out, n64) if want_f64 else (res_out, norm_out)
+
+
 def swiglu(a, b, cu_seqlens, cu_seqlens_padded, *, inner, a_row_stride=None, b_row_stride=None,
            out_row_stride=None, nrows=None, rows=None, out_init=None, want_f64=False, out=None):
     """out = silu(a) * b on valid rows.
@@ -233,3 +271,17 @@ def swiglu(a, b, cu_seqlens, cu_seqlens_padded, *, inner, a_row_stride=None, b_r
         _ptr(out, ctypes.c_uint16), ostride, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "swiglu")
     return (out, o64) if want_f64 else out
+
+
+def frames_to_u8(x, layout: int = 0) -> np.ndarray:
+    """fp32 frames [B, C, T, H, W] -> uint8 [B, T, H, W, C] (layout 0) or
+    [B, T, C, H, W] (layout 1)."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    if x.ndim != 5:
+        raise ValueError("expected [batch, channels, frames, height, width]")
+    B, C, T, H, W = x.shape
+    shape = (B, T, H, W, C) if layout == 0 else (B, T, C, H, W)
+    out = np.zeros(shape, dtype=np.uint8)
+    rc = lib().oracle_frames_to_u8(_ptr(x, ctypes.c_float), B, C, T, H, W, layout, _ptr(out, ctypes.c_uint8))
+    _check(rc, "frames_to_u8")
+    return out

@@ -328,6 +328,70 @@ int oracle_gated_residual(
     return 0;
 }
 
+/* ------------------------------------- gated residual + next adaLN */
+
+/* The residual update of one sublayer and the modulated normalization that
+ * opens the next one ("Why Real-Time MiniMax H3 Serving Requires More Than a
+ * Faster DiT", "Key takeaways", bullet 2 groups residual updates with
+ * modulation and normalization).  Step 1 is the gated residual, rounded to
+ * bf16 because that is the value the residual stream stores; step 2 is the
+ * adaLN modulation of those stored values. */
+int oracle_gated_residual_adaln(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const uint16_t* gate, int64_t gate_seq_stride,
+    const uint16_t* shift, const uint16_t* scale, int64_t mod_seq_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    if (!x || !y || !gate || !shift || !scale || !res_out || !norm_out || hidden <= 0)
+        return -1;
+    if (x_row_stride < hidden || y_row_stride < hidden || res_row_stride < hidden || norm_row_stride < hidden ||
+        gate_seq_stride < 0 || mod_seq_stride < 0)
+        return -1;
+    if (!seqlens_ok(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded))
+        return -1;
+    int64_t n = rows ? num_rows : num_rows_padded;
+
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t row = row_at(rows, i), r;
+        int32_t b;
+        if (row < 0 || row >= num_rows_padded)
+            continue;
+        if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
+            continue;
+        const uint16_t* g = gate + (int64_t)b * gate_seq_stride;
+        uint16_t* rr = res_out + row * res_row_stride;
+        /* step 1: residual update, stored as bf16 */
+        for (int32_t c = 0; c < hidden; ++c) {
+            double v = ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]);
+            rr[c] = oracle_f64_to_bf16(v);
+        }
+        /* step 2: adaLN of the stored residual */
+        const uint16_t* sh = shift + (int64_t)b * mod_seq_stride;
+        const uint16_t* sc = scale + (int64_t)b * mod_seq_stride;
+        double mean = 0.0;
+        for (int32_t c = 0; c < hidden; ++c)
+            mean += ld(&rr[c]);
+        mean /= (double)hidden;
+        double var = 0.0;
+        for (int32_t c = 0; c < hidden; ++c)
+            var += (ld(&rr[c]) - mean) * (ld(&rr[c]) - mean);
+        var /= (double)hidden;
+        double inv_std = 1.0 / sqrt(var + eps);
+        for (int32_t c = 0; c < hidden; ++c) {
+            double xhat = (ld(&rr[c]) - mean) * inv_std;
+            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);
+            put(norm_out, norm_out_f64, row * norm_row_stride + c, v);
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------- SwiGLU */
 
 int oracle_swiglu(
@@ -360,6 +424,48 @@ int oracle_swiglu(
             double silu = av / (1.0 + exp(-av));
             put(out, out_f64, row * out_row_stride + c, silu * bv);
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------ frames -> uint8 */
+
+/* "Why Real-Time MiniMax H3 Serving Requires More Than a Faster DiT", "Key
+ * takeaways", bullet 3: decoded frames are converted on the GPU into compact
+ * uint8 BTHWC data once, and the encoder reads planar paths from it.  The page
+ * gives no value mapping; the reading taken is the usual one for decoder
+ * output in [-1, 1]: scale to [0, 255], clamp, round to nearest even. */
+static uint8_t frame_value_to_u8(float x)
+{
+    float t = x + 1.0f;
+    float u = t * 127.5f;
+    if (!(u > 0.0f)) /* also NaN */
+        return 0;
+    if (u >= 255.0f)
+        return 255;
+    return (uint8_t)nearbyintf(u);
+}
+
+int oracle_frames_to_u8(const float* x, int64_t batch, int64_t channels, int64_t frames, int64_t height,
+                        int64_t width, int32_t layout, uint8_t* out)
+{
+    if (!x || !out || batch < 0 || channels < 0 || frames < 0 || height < 0 || width < 0)
+        return -1;
+    if (layout != 0 && layout != 1)
+        return -1;
+    int64_t planes = batch * frames;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bt = 0; bt < planes; ++bt) {
+        int64_t b = bt / frames, t = bt % frames;
+        for (int64_t c = 0; c < channels; ++c)
+            for (int64_t h = 0; h < height; ++h)
+                for (int64_t w = 0; w < width; ++w) {
+                    int64_t src = (((b * channels + c) * frames + t) * height + h) * width + w;
+                    int64_t dst = layout == 0
+                        ? (((b * frames + t) * height + h) * width + w) * channels + c
+                        : (((b * frames + t) * channels + c) * height + h) * width + w;
+                    out[dst] = frame_value_to_u8(x[src]);
+                }
     }
     return 0;
 }

@@ -89,6 +89,22 @@ int oracle_gated_residual(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows);
 
+/* Gated residual update followed by the next sublayer's adaLN, as one op:
+ *   res_out  = bf16(x + gate_b * y)                      (the updated residual stream)
+ *   norm_out = bf16(LN(res_out) * (1 + scale_b) + shift_b)
+ * LN reads the residual as stored (bf16), so the pair equals
+ * oracle_gated_residual followed by oracle_adaln_modulate on its output. */
+int oracle_gated_residual_adaln(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const uint16_t* gate, int64_t gate_seq_stride,
+    const uint16_t* shift, const uint16_t* scale, int64_t mod_seq_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows);
+
 /* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)). */
 int oracle_swiglu(
     const uint16_t* a, int64_t a_row_stride,
@@ -97,6 +113,18 @@ int oracle_swiglu(
     int32_t num_seqs, int64_t num_rows_padded, int32_t inner,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows);
+
+/* Decoded video frames -> uint8, converted once on the device before the
+ * media encoder.  x: fp32 [batch][channels][frames][height][width]
+ * (channels first, contiguous).  Each value becomes
+ *   u = rint(clamp((x + 1) * 127.5, 0, 255))
+ * in fp32 arithmetic, one IEEE operation at a time (x + 1, then * 127.5),
+ * ties to even, NaN -> 0.  The float decides an integer here, so this function
+ * computes in fp32 exactly as the device does, not in fp64.
+ * layout 0: out [batch][frames][height][width][channels]  (interleaved, "BTHWC")
+ * layout 1: out [batch][frames][channels][height][width]  (one plane per channel) */
+int oracle_frames_to_u8(const float* x, int64_t batch, int64_t channels, int64_t frames, int64_t height,
+                        int64_t width, int32_t layout, uint8_t* out);
 
 /* Number of OpenMP threads the oracle's row loops use (1 without OpenMP). */
 int oracle_num_threads(void);

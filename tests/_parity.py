@@ -83,6 +83,20 @@ def gpu_residual(w, inp, in_place=False):
     return out
 
 
+def gpu_fused(w, inp, in_place=False):
+    """Gated residual (gate = mod[:, 2]) fused with the MLP sublayer's adaLN
+    (shift = mod[:, 3], scale = mod[:, 4]); returns (res, norm) buffers."""
+    cs, cp, _ = device_packing(w)
+    x = inp["x"].cuda()
+    y = inp["y"].cuda()
+    mod = inp["mod"].cuda()
+    res = x if in_place else inp["out"].cuda()
+    norm = W.sentinel_like(inp["out"].shape).cuda()
+    dit.dit_gated_residual_adaln(W.rows_view(x), W.rows_view(y), mod[:, 2], mod[:, 3], mod[:, 4], cs, cp,
+                                 res_out=W.rows_view(res), norm_out=W.rows_view(norm), eps=w.eps)
+    return res, norm
+
+
 def gpu_swiglu(w, inp):
     cs, cp, _ = device_packing(w)
     ab = W.rows_view(inp["ab"].cuda())
@@ -116,6 +130,16 @@ def oracle_residual(w, inp, rows):
     flat = np.ascontiguousarray(tbits(inp["mod"]).reshape(-1))
     return oracle.gated_residual(x, y, flat[2 * w.hidden:], w.cu_seqlens, w.cu_seqlens_padded,
                                  hidden=w.hidden, gate_seq_stride=6 * w.hidden, rows=rows)
+
+
+def oracle_fused(w, inp, rows):
+    x = tbits(W.rows_view(inp["x"]))
+    y = tbits(W.rows_view(inp["y"]))
+    flat = np.ascontiguousarray(tbits(inp["mod"]).reshape(-1))
+    C = w.hidden
+    return oracle.gated_residual_adaln(x, y, flat[2 * C:], flat[3 * C:], flat[4 * C:], w.cu_seqlens,
+                                       w.cu_seqlens_padded, hidden=C, eps=w.eps, gate_seq_stride=6 * C,
+                                       mod_seq_stride=6 * C, rows=rows)
 
 
 def oracle_swiglu(w, inp, rows):

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 8, names
+    assert len(names) == 10, names
     for n in names:
         assert hasattr(L, n), n
     assert L.dit_abi_version() == 1
@@ -114,6 +114,31 @@ def test_residual_and_swiglu_argument_checks(L):
     assert sw(b=None) == NULL and sw(o=None) == NULL
     assert sw(os=32) == SHAPE and sw(I=0) == SHAPE
     assert sw(b=P + 64 * 2 + 2) == ALIGN and sw(as_=132) == ALIGN
+
+
+def test_fused_residual_adaln_argument_checks(L):
+    def call(**kw):
+        a = dict(x=P, xs=64, y=P, ys=64, g=P, gs=64, sh=P, sc=P, ms=64, r=P, rs=64, n=P, ns=64, B=1, rows=4,
+                 C=64, eps=1e-6)
+        a.update(kw)
+        return L.dit_gated_residual_adaln(a["x"], a["xs"], a["y"], a["ys"], a["g"], a["gs"], a["sh"], a["sc"],
+                                          a["ms"], a["r"], a["rs"], a["n"], a["ns"], P, P, a["B"], a["rows"],
+                                          a["C"], a["eps"], None)
+    assert call(n=None) == NULL and call(sh=None) == NULL and call(g=None) == NULL
+    assert call(ns=32) == SHAPE and call(ms=-8) == SHAPE and call(eps=-1.0) == SHAPE
+    assert call(C=16392, xs=16392, ys=16392, rs=16392, ns=16392) == UNSUP
+    assert call(r=P + 8) == ALIGN and call(gs=12) == ALIGN
+    assert call(B=0, x=None, n=None) == OK
+
+
+def test_frames_argument_checks(L):
+    assert L.dit_frames_to_u8(P, 1, 3, 2, 4, 16, 2, P, None) == UNSUP
+    assert L.dit_frames_to_u8(P, 1, -3, 2, 4, 16, 0, P, None) == SHAPE
+    assert L.dit_frames_to_u8(None, 1, 3, 2, 4, 16, 0, P, None) == NULL
+    assert L.dit_frames_to_u8(P, 1, 3, 2, 4, 16, 0, None, None) == NULL
+    assert L.dit_frames_to_u8(P + 2, 1, 3, 2, 4, 16, 0, P, None) == ALIGN
+    assert L.dit_frames_to_u8(None, 0, 3, 2, 4, 16, 0, None, None) == OK    # empty
+    assert L.dit_frames_to_u8(P, 1 << 40, 1 << 20, 1, 1, 1, 0, P, None) == SHAPE
 
 
 def test_validate_argument_checks(L):

@@ -58,6 +58,14 @@ def all_ops_full(w, in_place=False):
     P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, inp, rows)[rows], "swiglu")
     P.assert_untouched(out, inp["out"], keep, "swiglu")
 
+    inp = W.residual_inputs(w)
+    res, norm = P.gpu_fused(w, inp, in_place=in_place)
+    r_ref, n_ref = P.oracle_fused(w, inp, rows)
+    P.assert_close(P.gather_rows(res, rows), r_ref[rows], "fused residual")
+    P.assert_close(P.gather_rows(norm, rows), n_ref[rows], "fused norm")
+    P.assert_untouched(res, inp["x"] if in_place else inp["out"], keep, "fused residual")
+    P.assert_untouched(norm, inp["out"], keep, "fused norm")
+
 
 @pytest.mark.parametrize("in_place", [False, True])
 def test_ragged_batch(in_place):
@@ -125,6 +133,11 @@ def test_adaln_every_team_shape(hidden):
     out = P.gpu_adaln(w, inp)
     P.assert_close(P.gather_rows(out, rows), P.oracle_adaln(w, inp, rows)[rows], f"adaln {hidden}")
     P.assert_untouched(out, inp["out"], P.untouched_rows(w), "adaln")
+    inp = W.residual_inputs(w)
+    res, norm = P.gpu_fused(w, inp)
+    r_ref, n_ref = P.oracle_fused(w, inp, rows)
+    P.assert_close(P.gather_rows(res, rows), r_ref[rows], f"fused residual {hidden}")
+    P.assert_close(P.gather_rows(norm, rows), n_ref[rows], f"fused norm {hidden}")
 
 
 def test_swiglu_extreme_activations():

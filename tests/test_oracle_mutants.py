@@ -16,7 +16,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
-        "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py"]
+        "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py"]
 
 # (name, original text, planted mistake)
 MUTANTS = [
@@ -41,6 +41,10 @@ MUTANTS = [
      "double silu = bv / (1.0 + exp(-bv));\n            put(out, out_f64, row * out_row_stride + c, silu * av);"),
     ("bf16_truncates", "nearbyint(ax / spacing)", "floor(ax / spacing)"),
     ("padding_row_read", "if (r < len) {", "if (r <= len) {"),
+    ("fused_mean_over_x_not_residual", "mean += ld(&rr[c]);", "mean += ld(&x[row * x_row_stride + c]);"),
+    ("fused_residual_not_rounded_before_norm",
+     "double xhat = (ld(&rr[c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out",
+     "double xhat = (ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out"),
     ("rows_located_by_valid_offsets", "if (row >= cu_seqlens_padded[b] && row < cu_seqlens_padded[b + 1]) {",
      "if (row >= cu_seqlens[b] && row < cu_seqlens[b + 1]) {"),
 ]

@@ -76,3 +76,24 @@ def test_swiglu(case):
     P.assert_untouched(out, inp["out"], P.untouched_rows(w), f"{w.name} swiglu out")
     out2 = P.gpu_swiglu(w, inp)
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+def test_gated_residual_adaln(case):
+    w, inp, rows = case[0], case[1]["residual"], case[2]
+    res, norm = P.gpu_fused(w, inp)
+    torch.cuda.synchronize()
+    r_ref, n_ref = P.oracle_fused(w, inp, rows)
+    P.assert_close(P.gather_rows(res, rows), r_ref[rows], f"{w.name} fused residual")
+    P.assert_close(P.gather_rows(norm, rows), n_ref[rows], f"{w.name} fused norm")
+    keep = P.untouched_rows(w)
+    P.assert_untouched(res, inp["out"], keep, f"{w.name} fused res")
+    P.assert_untouched(norm, inp["out"], keep, f"{w.name} fused norm")
+    # the fused op reproduces the two separate kernels bit for bit
+    import dit_token_b200 as dit
+    cs, cp, _ = P.device_packing(w)
+    mod = inp["mod"].cuda()
+    r2 = P.gpu_residual(w, inp)
+    n2 = W.sentinel_like(inp["out"].shape).cuda()
+    dit.dit_adaln_modulate(W.rows_view(r2), mod[:, 3], mod[:, 4], cs, cp, out=W.rows_view(n2), eps=w.eps)
+    assert torch.equal(res.view(torch.int16), r2.view(torch.int16))
+    assert torch.equal(norm.view(torch.int16), n2.view(torch.int16))
