@@ -39,6 +39,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_qk_rmsnorm_rope.argtypes = [
             u16p, i64, u16p, i64, u16p, u16p, i32p, i32p, i32, i64, i32, i32, i32,
             i32p, i32, i32, i32, f64, f64, u16p, u16p, f64p, f64p, i64p, i64]
+        L.oracle_qk_rmsnorm_rope_ex.argtypes = [
+            u16p, i64, u16p, i64, u16p, u16p, i32p, i32p, i32, i64, i32, i32, i32,
+            i32p, i32, i32, i32, f64, f64, i32, u16p, u16p, f64p, f64p, i64p, i64]
         L.oracle_adaln_modulate.argtypes = [
             u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
         L.oracle_gated_residual.argtypes = [
@@ -50,7 +53,8 @@ def lib() -> ctypes.CDLL:
             u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
         L.oracle_frames_to_u8.argtypes = [ctypes.POINTER(ctypes.c_float), i64, i64, i64, i64, i64, i32,
                                           ctypes.POINTER(ctypes.c_uint8)]
-        for name in ("oracle_qk_rmsnorm_rope", "oracle_adaln_modulate", "oracle_frames_to_u8",
+        for name in ("oracle_qk_rmsnorm_rope", "oracle_qk_rmsnorm_rope_ex", "oracle_adaln_modulate",
+                     "oracle_frames_to_u8",
                      "oracle_gated_residual", "oracle_gated_residual_adaln", "oracle_swiglu",
                      "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
@@ -125,8 +129,12 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
                     num_q_heads, num_k_heads, head_dim, rope_grid=None,
                     sections=(0, 0, 0), rope_theta=10000.0, eps=1e-6,
                     q_row_stride=None, k_row_stride=None, rows=None,
-                    q_out_init=None, k_out_init=None, want_f64=False, q_out=None, k_out=None):
+                    q_out_init=None, k_out_init=None, want_f64=False, q_out=None, k_out=None,
+                    rope_mode="interleaved"):
     """Per-head Q/K RMSNorm fused with 1D / 3D rotary embedding.
+
+    rope_mode: "interleaved" (pairs 2j, 2j+1), "half" (pairs j, j + D/2) or
+    "none" (RMSNorm only).
 
     q, k: uint16 arrays whose first axis is the padded row; row strides
     default to the product of the remaining axes.  Returns (q_out, k_out) or,
@@ -147,12 +155,13 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
     wk = np.ascontiguousarray(_u16(k_weight))
     r, nr = _rows(rows)
     L = lib()
-    rc = L.oracle_qk_rmsnorm_rope(
+    mode = {"interleaved": 0, "half": 1, "none": 2}[rope_mode]
+    rc = L.oracle_qk_rmsnorm_rope_ex(
         _ptr(q, ctypes.c_uint16), qs, _ptr(k, ctypes.c_uint16), ks,
         _ptr(wq, ctypes.c_uint16), _ptr(wk, ctypes.c_uint16),
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows,
         num_q_heads, num_k_heads, head_dim,
-        _ptr(grid, ctypes.c_int32), *[int(s) for s in sections], float(rope_theta), float(eps),
+        _ptr(grid, ctypes.c_int32), *[int(s) for s in sections], float(rope_theta), float(eps), mode,
         _ptr(q_out, ctypes.c_uint16), _ptr(k_out, ctypes.c_uint16),
         _ptr(q64, ctypes.c_double), _ptr(k64, ctypes.c_double),
         _ptr(r, ctypes.c_int64), nr)

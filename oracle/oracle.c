@@ -144,14 +144,16 @@ static double rope_angle(int j, int head_dim, int is3d, const int64_t pos3[3], i
 }
 
 /* One head: RMSNorm over head_dim, times the weight, then rotate every
- * interleaved pair (2j, 2j+1) by its angle:
+ * pair of elements (i0, i1) of pair index j by its angle:
  *   ms    = (1/D) * sum_i x_i^2
  *   y_i   = x_i / sqrt(ms + eps) * w_i
- *   o_2j   = y_2j cos(a_j) - y_2j+1 sin(a_j)
- *   o_2j+1 = y_2j sin(a_j) + y_2j+1 cos(a_j) */
+ *   o_i0  = y_i0 cos(a_j) - y_i1 sin(a_j)
+ *   o_i1  = y_i0 sin(a_j) + y_i1 cos(a_j)
+ * Pair j is (2j, 2j+1) for interleaved rotary embedding, (j, j + D/2) for the
+ * half-split ("rotate half") layout; with no rotary embedding o = y. */
 static void rmsnorm_rope_head(const uint16_t* x, const uint16_t* w, int D, double eps,
                               int is3d, const int64_t pos3[3], int64_t pos1,
-                              const int32_t sec[3], double theta,
+                              const int32_t sec[3], double theta, int rope_mode,
                               uint16_t* out_bits, double* out_f64, double* y)
 {
     double ms = 0.0;
@@ -161,12 +163,19 @@ static void rmsnorm_rope_head(const uint16_t* x, const uint16_t* w, int D, doubl
     double inv_rms = 1.0 / sqrt(ms + eps);
     for (int i = 0; i < D; ++i)
         y[i] = ld(&x[i]) * inv_rms * ld(&w[i]);
+    if (rope_mode == ORACLE_ROPE_NONE) {
+        for (int i = 0; i < D; ++i)
+            put(out_bits, out_f64, i, y[i]);
+        return;
+    }
     for (int j = 0; j < D / 2; ++j) {
         double a = rope_angle(j, D, is3d, pos3, pos1, sec, theta);
         double c = cos(a), s = sin(a);
-        double y0 = y[2 * j], y1 = y[2 * j + 1];
-        put(out_bits, out_f64, 2 * j, y0 * c - y1 * s);
-        put(out_bits, out_f64, 2 * j + 1, y0 * s + y1 * c);
+        int i0 = rope_mode == ORACLE_ROPE_HALF ? j : 2 * j;
+        int i1 = rope_mode == ORACLE_ROPE_HALF ? j + D / 2 : 2 * j + 1;
+        double y0 = y[i0], y1 = y[i1];
+        put(out_bits, out_f64, i0, y0 * c - y1 * s);
+        put(out_bits, out_f64, i1, y0 * s + y1 * c);
     }
 }
 
@@ -182,7 +191,27 @@ int oracle_qk_rmsnorm_rope(
     uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_qk_rmsnorm_rope_ex(q, q_row_stride, k, k_row_stride, q_weight, k_weight, cu_seqlens,
+                                     cu_seqlens_padded, num_seqs, num_rows_padded, num_q_heads, num_k_heads,
+                                     head_dim, rope_grid, sec_t, sec_h, sec_w, rope_theta, eps,
+                                     ORACLE_ROPE_INTERLEAVED, q_out, k_out, q_out_f64, k_out_f64, rows, num_rows);
+}
+
+int oracle_qk_rmsnorm_rope_ex(
+    const uint16_t* q, int64_t q_row_stride,
+    const uint16_t* k, int64_t k_row_stride,
+    const uint16_t* q_weight, const uint16_t* k_weight,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded,
+    int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+    const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+    double rope_theta, double eps, int32_t rope_mode,
+    uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!q || !k || !q_weight || !k_weight || !q_out || !k_out)
+        return -1;
+    if (rope_mode != ORACLE_ROPE_INTERLEAVED && rope_mode != ORACLE_ROPE_HALF && rope_mode != ORACLE_ROPE_NONE)
         return -1;
     if (head_dim <= 0 || head_dim % 2 || head_dim > 1024 || num_q_heads < 0 || num_k_heads < 0)
         return -1;
@@ -230,12 +259,12 @@ int oracle_qk_rmsnorm_rope(
             }
             for (int32_t h = 0; h < num_q_heads; ++h) {
                 int64_t off = row * q_row_stride + (int64_t)h * head_dim;
-                rmsnorm_rope_head(q + off, q_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta,
+                rmsnorm_rope_head(q + off, q_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta, rope_mode,
                                   q_out + off, q_out_f64 ? q_out_f64 + off : NULL, y);
             }
             for (int32_t h = 0; h < num_k_heads; ++h) {
                 int64_t off = row * k_row_stride + (int64_t)h * head_dim;
-                rmsnorm_rope_head(k + off, k_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta,
+                rmsnorm_rope_head(k + off, k_weight, head_dim, eps, is3d, pos3, pos1, sec, rope_theta, rope_mode,
                                   k_out + off, k_out_f64 ? k_out_f64 + off : NULL, y);
             }
         }

@@ -68,6 +68,26 @@ int oracle_qk_rmsnorm_rope(
     uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
     const int64_t* rows, int64_t num_rows);
 
+/* The same with a choice of rotary layout:
+ *   ORACLE_ROPE_INTERLEAVED  pairs (2j, 2j+1)            (what oracle_qk_rmsnorm_rope does)
+ *   ORACLE_ROPE_HALF         pairs (j, j + head_dim/2)   ("rotate half" layout)
+ *   ORACLE_ROPE_NONE         no rotation: per-head RMSNorm times the weight only
+ * Pair j has the same angle in both rotary layouts. */
+#define ORACLE_ROPE_INTERLEAVED 0
+#define ORACLE_ROPE_HALF 1
+#define ORACLE_ROPE_NONE 2
+int oracle_qk_rmsnorm_rope_ex(
+    const uint16_t* q, int64_t q_row_stride,
+    const uint16_t* k, int64_t k_row_stride,
+    const uint16_t* q_weight, const uint16_t* k_weight,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded,
+    int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+    const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+    double rope_theta, double eps, int32_t rope_mode,
+    uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
+    const int64_t* rows, int64_t num_rows);
+
 /* Adaptive LayerNorm modulation: out = LN(x) * (1 + scale_b) + shift_b.
  * shift/scale: bf16[num_seqs][hidden] with a per-sequence stride of
  * mod_seq_stride elements. */

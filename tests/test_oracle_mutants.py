@@ -16,13 +16,18 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
-        "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py"]
+        "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py",
+        "tests/test_oracle_frames.py", "tests/test_oracle_rope_modes.py"]
 
 # (name, original text, planted mistake)
 MUTANTS = [
     ("rope_sign", "y0 * c - y1 * s", "y0 * c + y1 * s"),
-    ("rope_half_split_read", "double y0 = y[2 * j], y1 = y[2 * j + 1];",
-     "double y0 = y[j], y1 = y[j + D / 2];"),
+    ("rope_interleaved_read_as_half_split",
+     "int i0 = rope_mode == ORACLE_ROPE_HALF ? j : 2 * j;\n        int i1 = rope_mode == ORACLE_ROPE_HALF ? j + D / 2 : 2 * j + 1;",
+     "int i0 = j;\n        int i1 = j + D / 2;"),
+    ("rope_half_wrong_partner", "int i1 = rope_mode == ORACLE_ROPE_HALF ? j + D / 2 : 2 * j + 1;",
+     "int i1 = rope_mode == ORACLE_ROPE_HALF ? D - 1 - j : 2 * j + 1;"),
+    ("rope_none_drops_weight", "put(out_bits, out_f64, i, y[i]);", "put(out_bits, out_f64, i, ld(&x[i]) * inv_rms);"),
     ("rms_eps_dropped", "sqrt(ms + eps)", "sqrt(ms)"),
     ("rms_mean_not_divided", "ms /= (double)D;", ""),
     ("rms_weight_dropped", "y[i] = ld(&x[i]) * inv_rms * ld(&w[i]);", "y[i] = ld(&x[i]) * inv_rms;"),
@@ -45,6 +50,10 @@ MUTANTS = [
     ("fused_residual_not_rounded_before_norm",
      "double xhat = (ld(&rr[c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out",
      "double xhat = (ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out"),
+    ("frames_truncates", "return (uint8_t)nearbyintf(u);", "return (uint8_t)u;"),
+    ("frames_no_clamp_top", "if (u >= 255.0f)\n        return 255;", ""),
+    ("frames_wrong_layout", "? (((b * frames + t) * height + h) * width + w) * channels + c",
+     "? (((b * frames + t) * width + w) * height + h) * channels + c"),
     ("rows_located_by_valid_offsets", "if (row >= cu_seqlens_padded[b] && row < cu_seqlens_padded[b + 1]) {",
      "if (row >= cu_seqlens[b] && row < cu_seqlens[b + 1]) {"),
 ]
