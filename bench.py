@@ -546,6 +546,34 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_table(args):
+    """Per-op table over every workload (markdown on stdout): the measured
+    results that complement the single JSON line."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from dit_token_b200 import build
+    build.build()
+    peak, kind = measured_peak()
+    print(f"| workload | op | GPU us | tokens/s | GB/s | % of 8 TB/s | % of {kind} {peak:.0f} GB/s |")
+    print("|---|---|---|---|---|---|---|")
+    for name in W.WORKLOAD_NAMES:
+        w = W.workload(name, args.seed)
+        host = host_inputs(w)
+        step = Step(w, host, device)
+        _, op_ms, _ = time_device(step, args.steps, args.warmup, device)
+        nxt = time_next_ops(step, args.steps, args.warmup, device)
+        ab = algorithmic_bytes(w)
+        ab["gated_residual_adaln"] = 8 * w.hidden * w.num_valid
+        op_ms.update(nxt)
+        for op in list(OPS) + ["gated_residual_adaln"]:
+            us = op_ms[op] * 1e3
+            gbs = ab[op] / (us * 1e-6) / 1e9
+            print(f"| {name} | {op} | {us:.1f} | {w.num_valid / (us * 1e-6):.3g} | {gbs:.0f} | "
+                  f"{100 * gbs / 8000:.1f} | {100 * gbs / peak:.1f} |", flush=True)
+        del step, host
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -560,6 +588,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", action="store_true",
+                    help="print a per-op markdown table over every workload instead of the JSON line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -567,7 +597,9 @@ def main(argv=None):
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
-    if args.impl == "reference":
+    if args.table:
+        run_table(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_dit(args)

@@ -55,6 +55,8 @@ _F32 = ctypes.c_float
 _SIGNATURES = {
     "dit_qk_rmsnorm_rope": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
                             _VP, _I32, _I32, _I32, _F32, _F32, _VP],
+    "dit_qk_rmsnorm_rope_ex": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
+                               _VP, _I32, _I32, _I32, _F32, _F32, _I32, _VP],
     "dit_adaln_modulate": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _VP],
     "dit_gated_residual": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
     "dit_swiglu": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
@@ -149,12 +151,15 @@ def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor
                         num_q_heads: int, num_k_heads: int, head_dim: int,
                         rope_grid: Optional[torch.Tensor] = None,
                         sections: Sequence[int] = (0, 0, 0), rope_theta: float = 10000.0,
-                        eps: float = 1e-6, stream=None) -> None:
+                        eps: float = 1e-6, rope_mode: str = "interleaved", stream=None) -> None:
     """In place: q, k <- RoPE(RMSNorm_head(q) * q_weight), RoPE(RMSNorm_head(k) * k_weight).
 
     q: [rows, num_q_heads * head_dim] (or [rows, heads, head_dim]) bf16, any
     row stride; k likewise.  rope_grid: int32 [num_seqs, 3] (T, H, W) or None
-    (every row 1D); sections: t/h/w widths of head_dim on 3D rows."""
+    (every row 1D); sections: t/h/w widths of head_dim on 3D rows.
+    rope_mode: "interleaved" (pairs 2j, 2j+1; the C entry dit_qk_rmsnorm_rope),
+    "half" (pairs j, j + D/2) or "none" (RMSNorm only) -- the latter two, and
+    head_dim 256, go through dit_qk_rmsnorm_rope_ex."""
     qp, qs = _rows(q, "q")
     kp, ks = _rows(k, "k")
     if k.size(0) != q.size(0):
@@ -167,9 +172,13 @@ def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor
             raise TypeError("rope_grid: expected a contiguous int32 CUDA tensor [num_seqs, 3]")
         gp = rope_grid.data_ptr()
     st, sh, sw = (int(s) for s in sections)
-    _call("dit_qk_rmsnorm_rope", qp, qs, kp, ks, _vec(q_weight, "q_weight"), _vec(k_weight, "k_weight"),
-          cs, cp, B, q.size(0), num_q_heads, num_k_heads, head_dim, gp or None, st, sh, sw,
-          float(rope_theta), float(eps), _stream(stream))
+    args = (qp, qs, kp, ks, _vec(q_weight, "q_weight"), _vec(k_weight, "k_weight"), cs, cp, B, q.size(0),
+            num_q_heads, num_k_heads, head_dim, gp or None, st, sh, sw, float(rope_theta), float(eps))
+    mode = {"interleaved": 0, "half": 1, "none": 2}[rope_mode]
+    if mode == 0 and head_dim in (64, 128):
+        _call("dit_qk_rmsnorm_rope", *args, _stream(stream))
+    else:
+        _call("dit_qk_rmsnorm_rope_ex", *args, mode, _stream(stream))
 
 
 def dit_adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,

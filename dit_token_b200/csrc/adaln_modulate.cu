@@ -1,102 +1,270 @@
 // adaln_modulate.cu -- out = LN(x) * (1 + scale_b) + shift_b over the valid rows
 // of a packed sequence ("Why Real-Time MiniMax H3 Serving Requires More Than a
 // Faster DiT", "Key takeaways", bullet 2: the adaptive normalization and its
-// modulation are one of the fused operators).  LN has no affine; the variance is the biased one.
+// modulation are one of the fused operators).  LN has no affine; the variance
+// is the biased one.
 //
-// A team of TEAM warps owns one row and keeps the whole row in registers
-// (VPT 16-byte vectors per lane), so x is read from HBM once: a warp-shuffle
-// sum gives the mean, a second pass over the registers the sum of squared
-// deviations (exact two-pass variance), and a third pass writes the
-// modulated output.  Teams of more than one warp combine their partial sums
-// through shared memory behind a named barrier of their own, so the teams of
-// a CTA run independently.  The register budget is capped so that enough
-// CTAs stay resident to keep ~10 rows of loads in flight per SM: the kernel
-// is bound by bytes in flight, not by arithmetic.  HBM traffic: 4 bytes per
-// element.
+// Why this shape.  With only 4 bytes of HBM traffic per element, this op is
+// paced by instruction issue, not by HBM, unless every per-row and
+// per-element cost is cut (ncu on a team-per-row kernel: 20.6 thread
+// instructions per element, 70 % of issue slots busy, 48 % of DRAM peak; the
+// per-row costs -- finding the row, merging statistics across warps -- were
+// ~450 instructions per warp-row).  So, for rows of up to 6144 elements:
+//  * one warp owns a whole row (VPT 16-byte vectors per lane, x read from HBM
+//    once and kept in registers); no cross-warp merge, no barrier per row;
+//  * persistent CTAs of 8 warps, each warp walking a contiguous run of valid
+//    rows: the row mapping advances incrementally instead of being searched;
+//  * the modulation of the (at most two) sequences a CTA touches is staged
+//    once in shared memory as fp32 A = 1 + scale and B = shift, so the output
+//    pass is (x * rstd - mean * rstd) * A + B with packed fp32 FMAs and no
+//    per-row unpacking of the vectors (rows of any third sequence read them
+//    from global memory instead);
+//  * statistics in one pass (per-lane shifted sums merged as count/mean/M2
+//    moments by warp shuffles), arithmetic on packed fp32 pairs.
+// Wider rows (up to 16384) use a team of 2-8 warps per row with the same
+// statistics and a named barrier per team.  HBM traffic: 4 bytes per element.
+//
+// Measured alternatives (batched varlen, hidden 5120, 1.43 GB per launch):
+// team of 4 warps per row 299 us; 2 warps 263 us; CTA-wide smem ring fed by
+// cp.async 370-450 us; persistent 4-warp CTAs with 3 rows prefetched in
+// registers 352 us; the row streamed twice (second read from L2) 339 us;
+// this kernel 257 us.
 #include "common.cuh"
 #include "launch.h"
 
 namespace dit {
 namespace {
 
+constexpr int kMaxWarpVpt = 24;    // widest row a single warp holds: 24 * 256 = 6144 elements
+constexpr int kSmemBudget = 104 * 1024;
+
+// Statistics of the VPT vectors a lane holds (vectors past nvec are empty),
+// merged over the warp.  Vector i of the lane is vector i * STRIDE + lane_vec0
+// of the row.
+template <int VPT, int STRIDE>
+__device__ __forceinline__ Moments lane_row_moments(const uint4 (&xv)[VPT], int lane_vec0, int nvec)
+{
+    const float k = bf16_lo(xv[0].x);
+    const f32x2 kk = f2_make(k, k);
+    f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
+    float cnt = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        if (i * STRIDE + lane_vec0 < nvec) {
+            const uint32_t w[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const f32x2 d = f2_sub(f2_from_bf16x2(w[e]), kk);
+                s2 = f2_add(s2, d);
+                q2 = f2_fma(d, d, q2);
+            }
+            cnt += 8.f;
+        }
+    }
+    return moments_warp(moments_from_sums(cnt, k, s2.x + s2.y, q2.x + q2.y));
+}
+
+// One output vector: (x * rstd + nb) * A + B for the 8 elements of x.
+__device__ __forceinline__ uint4 modulate8(uint4 x, f32x2 r2, f32x2 b2, const f32x2 (&A)[4], const f32x2 (&B)[4])
+{
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        o[e] = f2_to_bf16x2(f2_fma(f2_fma(f2_from_bf16x2(w[e]), r2, b2), A[e], B[e]));
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// A = 1 + scale and B = shift of vector j, from global bf16.
+__device__ __forceinline__ void mod_from_global(const uint16_t* sh, const uint16_t* sc, int j, f32x2 (&A)[4],
+                                                f32x2 (&B)[4])
+{
+    const uint4 shv = ld_shared_vec(sh + 8 * j);
+    const uint4 scv = ld_shared_vec(sc + 8 * j);
+    const uint32_t hw[4] = {shv.x, shv.y, shv.z, shv.w};
+    const uint32_t cw[4] = {scv.x, scv.y, scv.z, scv.w};
+    const f32x2 one2 = f2_make(1.f, 1.f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        A[e] = f2_add(f2_from_bf16x2(cw[e]), one2);
+        B[e] = f2_from_bf16x2(hw[e]);
+    }
+}
+
+// ------------------------------------------------------------ warp per row
+
+template <int VPT>
+__global__ void __launch_bounds__(kCtaThreads)
+adaln_warp_kernel(const AdalnParams p, int slots)
+{
+    extern __shared__ __align__(16) float mod_smem[];  // [slots][2][hidden]: A, then B
+    const int nvec = p.hidden / 8;
+    const int C = p.hidden;
+    const int tid = threadIdx.x;
+    const int lane = tid & (kWarp - 1), warp = tid >> 5;
+
+    // this CTA's contiguous run of valid-row ordinals, then this warp's share
+    const int total = min(max(__ldg(p.pk.cu_seqlens + p.pk.num_seqs), 0), p.pk.num_rows_padded);
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int c0 = min(total, (int)blockIdx.x * per);
+    const int c1 = min(total, c0 + per);
+    if (c1 <= c0)
+        return;  // uniform over the CTA
+
+    // stage the modulation of the first and the last sequence of the run
+    int staged[2] = {-1, -1};
+    {
+        const int b0 = find_seq(c0, p.pk.cu_seqlens, p.pk.num_seqs, lane);
+        const int b1 = find_seq(c1 - 1, p.pk.cu_seqlens, p.pk.num_seqs, lane);
+        staged[0] = slots > 0 ? b0 : -1;
+        staged[1] = (slots > 1 && b1 != b0) ? b1 : -1;
+#pragma unroll
+        for (int sidx = 0; sidx < 2; ++sidx) {
+            const int b = staged[sidx];
+            if (b < 0)
+                continue;  // uniform
+            float* A = mod_smem + (size_t)sidx * 2 * C;
+            float* B = A + C;
+            const uint16_t* sh = p.shift + (int64_t)b * p.mod_seq_stride;
+            const uint16_t* sc = p.scale + (int64_t)b * p.mod_seq_stride;
+            for (int j = tid; j < nvec; j += kCtaThreads) {
+                float a[8], bb[8];
+                unpack8(ld_shared_vec(sc + 8 * j), a);
+                unpack8(ld_shared_vec(sh + 8 * j), bb);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    A[8 * j + e] = 1.0f + a[e];
+                    B[8 * j + e] = bb[e];
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    const int wper = (c1 - c0 + kWarpsPerCta - 1) / kWarpsPerCta;
+    const int w0 = min(c1, c0 + warp * wper);
+    const int w1 = min(c1, w0 + wper);
+    if (w1 <= w0)
+        return;  // no barrier follows
+    RowCursor cur{p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded};
+    {
+        const int b = find_seq(w0, p.pk.cu_seqlens, p.pk.num_seqs, lane);
+        cur.load(b < 0 ? 0 : b);
+    }
+    const float inv_n = 1.0f / (float)C;
+
+    for (int v = w0; v < w1; ++v) {
+        const int row = cur.row(v);
+        if (row < 0)
+            continue;  // uniform over the warp
+        const int seq = cur.b;
+        const uint16_t* xr = p.x + (int64_t)row * p.x_row_stride + 8 * lane;
+        uint4 xv[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            xv[i] = i * kWarp + lane < nvec ? ld_stream(xr + 8 * kWarp * i) : make_uint4(0u, 0u, 0u, 0u);
+
+        const Moments m = lane_row_moments<VPT, kWarp>(xv, lane, nvec);
+        const float rstd = rsqrtf(m.m2 * inv_n + p.eps);
+        const f32x2 r2 = f2_make(rstd, rstd);
+        const float nb = -m.mean * rstd;
+        const f32x2 b2 = f2_make(nb, nb);
+
+        uint16_t* orow = p.out + (int64_t)row * p.out_row_stride + 8 * lane;
+        const int sidx = seq == staged[0] ? 0 : (seq == staged[1] ? 1 : -1);
+        if (sidx >= 0) {
+            const float* A = mod_smem + (size_t)sidx * 2 * C + 8 * lane;
+            const float* B = A + C;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                if (i * kWarp + lane < nvec) {
+                    const float4* A4 = reinterpret_cast<const float4*>(A + 8 * kWarp * i);
+                    const float4* B4 = reinterpret_cast<const float4*>(B + 8 * kWarp * i);
+                    const float4 a0 = A4[0], a1 = A4[1], q0 = B4[0], q1 = B4[1];
+                    const f32x2 Av[4] = {f2_make(a0.x, a0.y), f2_make(a0.z, a0.w), f2_make(a1.x, a1.y),
+                                         f2_make(a1.z, a1.w)};
+                    const f32x2 Bv[4] = {f2_make(q0.x, q0.y), f2_make(q0.z, q0.w), f2_make(q1.x, q1.y),
+                                         f2_make(q1.z, q1.w)};
+                    st_stream(orow + 8 * kWarp * i, modulate8(xv[i], r2, b2, Av, Bv));
+                }
+            }
+        } else {
+            const uint16_t* sh = p.shift + (int64_t)seq * p.mod_seq_stride;
+            const uint16_t* sc = p.scale + (int64_t)seq * p.mod_seq_stride;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int j = i * kWarp + lane;
+                if (j < nvec) {
+                    f32x2 Av[4], Bv[4];
+                    mod_from_global(sh, sc, j, Av, Bv);
+                    st_stream(orow + 8 * kWarp * i, modulate8(xv[i], r2, b2, Av, Bv));
+                }
+            }
+        }
+    }
+}
+
+template <int VPT>
+cudaError_t launch_warp(const AdalnParams& p, cudaStream_t stream)
+{
+    const size_t slot_bytes = (size_t)2 * p.hidden * sizeof(float);
+    const int slots = 2 * slot_bytes <= (size_t)kSmemBudget ? 2 : (slot_bytes <= (size_t)kSmemBudget ? 1 : 0);
+    const size_t smem = slots * slot_bytes;
+    cudaError_t e;
+    if (smem > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(adaln_warp_kernel<VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+        return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_warp_kernel<VPT>, kCtaThreads, smem)) !=
+            cudaSuccess)
+        return e;
+    const long long want = (long long)sms * (per_sm > 0 ? per_sm : 1);
+    const long long rows_cap = (p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta;
+    const unsigned grid = (unsigned)(want < rows_cap ? want : rows_cap);
+    adaln_warp_kernel<VPT><<<grid, kCtaThreads, smem, stream>>>(p, slots);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ team per row
+
 template <int VPT, int TEAM>
 __global__ void __launch_bounds__(kCtaThreads, MinCtas<VPT>::value)
-adaln_kernel(const AdalnParams p)
+adaln_team_kernel(const AdalnParams p)
 {
     constexpr int kRowsPerCta = kWarpsPerCta / TEAM;
     constexpr int kTeamThreads = TEAM * kWarp;
-    __shared__ float red[2][kWarpsPerCta];
-
+    __shared__ Moments red[kWarpsPerCta];
     const int lane = threadIdx.x & (kWarp - 1);
     const int warp = threadIdx.x >> 5;
     const int team = warp / TEAM;
-    const int tt = (warp % TEAM) * kWarp + lane;  // thread index within the team
+    const int tt = (warp % TEAM) * kWarp + lane;
     const int v = blockIdx.x * kRowsPerCta + team;
     RowSlot s;
-    const bool active = map_valid_row(v, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs,
-                                      p.pk.num_rows_padded, lane, s);
-    if (!active)
-        return;  // the whole team leaves: its barriers involve only its own warps
+    if (!map_valid_row(v, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded, lane, s))
+        return;  // the whole team leaves: its barrier involves only its own warps
     const int nvec = p.hidden / 8;
     const uint16_t* xr = p.x + (int64_t)s.row * p.x_row_stride;
-
     uint4 xv[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         xv[i] = j < nvec ? ld_stream(xr + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
     }
-
-    // mean
-    float sum = 0.f;
+    Moments m = lane_row_moments<VPT, kTeamThreads>(xv, tt, nvec);
+    if (lane == 0)
+        red[warp] = m;
+    team_barrier<TEAM>(team);
+    m = red[team * TEAM];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        float f[8];
-        unpack8(xv[i], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            sum += f[e];
-    }
-    sum = group_sum<kWarp>(sum);
-    if (TEAM > 1) {
-        if (lane == 0)
-            red[0][warp] = sum;
-        team_barrier<TEAM>(team);
-        sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < TEAM; ++w)
-            sum += red[0][team * TEAM + w];
-    }
-    const float inv_n = 1.0f / (float)p.hidden;
-    const float mean = sum * inv_n;
-
-    // biased variance about the mean (padding lanes hold zeros: skip them)
-    float sq = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int j = i * kTeamThreads + tt;
-        if (j < nvec) {
-            float f[8];
-            unpack8_again(xv[i], f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = f[e] - mean;
-                sq = fmaf(d, d, sq);
-            }
-        }
-    }
-    sq = group_sum<kWarp>(sq);
-    if (TEAM > 1) {
-        if (lane == 0)
-            red[1][warp] = sq;
-        team_barrier<TEAM>(team);
-        sq = 0.f;
-#pragma unroll
-        for (int w = 0; w < TEAM; ++w)
-            sq += red[1][team * TEAM + w];
-    }
-    const float rstd = rsqrtf(sq * inv_n + p.eps);
-
+    for (int w = 1; w < TEAM; ++w)
+        m = moments_merge(m, red[team * TEAM + w]);
+    const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);
+    const f32x2 r2 = f2_make(rstd, rstd);
+    const float nb = -m.mean * rstd;
+    const f32x2 b2 = f2_make(nb, nb);
     const uint16_t* sh = p.shift + (int64_t)s.seq * p.mod_seq_stride;
     const uint16_t* sc = p.scale + (int64_t)s.seq * p.mod_seq_stride;
     uint16_t* orow = p.out + (int64_t)s.row * p.out_row_stride;
@@ -104,238 +272,26 @@ adaln_kernel(const AdalnParams p)
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
-            float f[8], shf[8], scf[8], o[8];
-            unpack8_again(xv[i], f);
-            unpack8(ld_shared_vec(sh + 8 * j), shf);
-            unpack8(ld_shared_vec(sc + 8 * j), scf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                o[e] = fmaf((f[e] - mean) * rstd, 1.0f + scf[e], shf[e]);
-            st_stream(orow + 8 * j, pack8(o));
+            f32x2 Av[4], Bv[4];
+            mod_from_global(sh, sc, j, Av, Bv);
+            st_stream(orow + 8 * j, modulate8(xv[i], r2, b2, Av, Bv));
         }
     }
-}
-
-// Pipelined variant: persistent CTAs, each owning one contiguous range of
-// valid-row ordinals.  An S-stage shared-memory ring filled by cp.async keeps
-// S - 1 rows per CTA in flight while the current row is reduced and written;
-// the ordinal -> padded-row mapping advances incrementally (global loads only
-// when a sequence boundary is crossed), and the current sequence's shift and
-// scale vectors sit in shared memory.  The whole CTA works on one row: two
-// block reductions (mean, then squared deviations), then the output pass.
-__device__ __forceinline__ float block_sum(float v, float* red, int warp, int lane)
-{
-    v = group_sum<kWarp>(v);
-    if (lane == 0)
-        red[warp] = v;
-    __syncthreads();
-    float t = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarpsPerCta; ++w)
-        t += red[w];
-    return t;
-}
-
-// Walks valid-row ordinals upward; every thread holds the same state.
-struct RowCursor {
-    const int32_t* cs;
-    const int32_t* cp;
-    int B;
-    int rows_padded;
-    int b;       // current sequence
-    int cs0, cs1, cp0, cp1;
-
-    __device__ void load(int bb)
-    {
-        b = bb;
-        cs0 = __ldg(cs + b);
-        cs1 = __ldg(cs + b + 1);
-        cp0 = __ldg(cp + b);
-        cp1 = __ldg(cp + b + 1);
-    }
-    // Padded row of ordinal v (v never decreases between calls), or -1.
-    __device__ int row(int v)
-    {
-        while (v >= cs1 && b + 1 < B)
-            load(b + 1);
-        const int r = v - cs0;
-        if (r < 0 || r >= cs1 - cs0 || r >= cp1 - cp0)
-            return -1;
-        const long long rr = (long long)cp0 + r;
-        return rr < rows_padded ? (int)rr : -1;
-    }
-};
-
-template <int S>
-__global__ void __launch_bounds__(kCtaThreads)
-adaln_pipelined_kernel(const AdalnParams p)
-{
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int nvec = p.hidden / 8;
-    uint4* stage = reinterpret_cast<uint4*>(smem_raw);  // [S][nvec]
-    uint4* mod_sh = stage + S * nvec;                    // shift of the current sequence
-    uint4* mod_sc = mod_sh + nvec;                       // scale of the current sequence
-    __shared__ float red[2][kWarpsPerCta];
-    __shared__ int slot_row[S];
-    __shared__ int slot_seq[S];
-
-    const int tid = threadIdx.x;
-    const int lane = tid & (kWarp - 1), warp = tid >> 5;
-    const int total = min(max(__ldg(p.pk.cu_seqlens + p.pk.num_seqs), 0), p.pk.num_rows_padded);
-    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int v0 = min(total, (int)blockIdx.x * per);
-    const int n = min(total, v0 + per) - v0;
-    if (n <= 0)
-        return;  // uniform: the whole CTA leaves before any barrier
-
-    RowCursor cur{p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded};
-    RowSlot first;
-    const bool ok0 = map_valid_row(v0, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs,
-                                   p.pk.num_rows_padded, lane, first);
-    cur.load(ok0 ? first.seq : 0);
-
-    auto issue = [&](int i) {
-        const int st = i % S;
-        const int row = cur.row(v0 + i);
-        if (tid == 0) {
-            slot_row[st] = row;
-            slot_seq[st] = cur.b;
-        }
-        if (row >= 0) {
-            const uint16_t* src = p.x + (int64_t)row * p.x_row_stride;
-            uint4* dst = stage + st * nvec;
-            for (int j = tid; j < nvec; j += kCtaThreads)
-                cp_async16(dst + j, src + 8 * j);
-        }
-        cp_async_commit();
-    };
-
-#pragma unroll
-    for (int i = 0; i < S - 1; ++i) {
-        if (i < n)
-            issue(i);
-        else
-            cp_async_commit();  // keep one group per ring slot
-    }
-    const float inv_n = 1.0f / (float)p.hidden;
-    int mod_seq = -1;
-    for (int i = 0; i < n; ++i) {
-        if (i + S - 1 < n)
-            issue(i + S - 1);
-        else
-            cp_async_commit();
-        cp_async_wait<S - 1>();  // this thread's copies of row i have landed
-        __syncthreads();         // ... and everyone else's
-        const int st = i % S;
-        const int row = slot_row[st];
-        if (row >= 0) {  // uniform across the CTA
-            const int seq = slot_seq[st];
-            if (seq != mod_seq) {  // uniform; rare (sequence boundary)
-                const uint16_t* sh = p.shift + (int64_t)seq * p.mod_seq_stride;
-                const uint16_t* sc = p.scale + (int64_t)seq * p.mod_seq_stride;
-                for (int j = tid; j < nvec; j += kCtaThreads) {
-                    mod_sh[j] = ld_shared_vec(sh + 8 * j);
-                    mod_sc[j] = ld_shared_vec(sc + 8 * j);
-                }
-                mod_seq = seq;
-                // visibility: the block_sum barriers below come before any read
-            }
-            const uint4* xs = stage + st * nvec;
-            float sum = 0.f;
-            for (int j = tid; j < nvec; j += kCtaThreads) {
-                float f[8];
-                unpack8(xs[j], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    sum += f[e];
-            }
-            const float mean = block_sum(sum, red[0], warp, lane) * inv_n;
-            float sq = 0.f;
-            for (int j = tid; j < nvec; j += kCtaThreads) {
-                float f[8];
-                unpack8(xs[j], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float d = f[e] - mean;
-                    sq = fmaf(d, d, sq);
-                }
-            }
-            const float rstd = rsqrtf(block_sum(sq, red[1], warp, lane) * inv_n + p.eps);
-            uint16_t* orow = p.out + (int64_t)row * p.out_row_stride;
-            for (int j = tid; j < nvec; j += kCtaThreads) {
-                float f[8], shf[8], scf[8], o[8];
-                unpack8(xs[j], f);
-                unpack8(mod_sh[j], shf);
-                unpack8(mod_sc[j], scf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    o[e] = fmaf((f[e] - mean) * rstd, 1.0f + scf[e], shf[e]);
-                st_stream(orow + 8 * j, pack8(o));
-            }
-        }
-        __syncthreads();  // ring slot st (and the shift/scale copy) may be rewritten next
-    }
-    cp_async_wait<0>();
-}
-
-template <int S>
-cudaError_t launch_pipelined(const AdalnParams& p, cudaStream_t stream)
-{
-    const size_t smem = (size_t)(S + 2) * (p.hidden / 8) * sizeof(uint4);
-    cudaError_t e = cudaFuncSetAttribute(adaln_pipelined_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess)
-        return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_pipelined_kernel<S>, kCtaThreads,
-                                                           smem)) != cudaSuccess)
-        return e;
-    const long long want = (long long)sms * (per_sm > 0 ? per_sm : 1);
-    const unsigned grid = (unsigned)(want < p.pk.num_rows_padded ? want : p.pk.num_rows_padded);
-    adaln_pipelined_kernel<S><<<grid, kCtaThreads, smem, stream>>>(p);
-    return cudaGetLastError();
-}
-
-#ifndef DIT_ADALN_PIPELINED
-#define DIT_ADALN_PIPELINED 0
-#endif
-#ifndef DIT_ADALN_MAX_VPT
-#define DIT_ADALN_MAX_VPT 8
-#endif
-
-// Vectors per lane that have an instantiation; a row needing another count
-// uses the next larger one (the extra slots are predicated off).
-constexpr int kVptSteps[] = {1, 2, 3, 4, 5, 6, 7, 8, 10, 12, 16, 20, 24};
-
-template <int TEAM, int VPT>
-void launch_one(const AdalnParams& p, cudaStream_t stream)
-{
-    const int rows_per_cta = kWarpsPerCta / TEAM;
-    const unsigned grid = (unsigned)((p.pk.num_rows_padded + rows_per_cta - 1) / rows_per_cta);
-    adaln_kernel<VPT, TEAM><<<grid, kCtaThreads, 0, stream>>>(p);
 }
 
 template <int TEAM>
-cudaError_t launch_team(const AdalnParams& p, int vpt, cudaStream_t stream)
+cudaError_t launch_team(const AdalnParams& p, cudaStream_t stream)
 {
+    const int nvec = p.hidden / 8;
+    const int vpt = (nvec + TEAM * kWarp - 1) / (TEAM * kWarp);
+    const int rows_per_cta = kWarpsPerCta / TEAM;
+    const unsigned grid = (unsigned)((p.pk.num_rows_padded + rows_per_cta - 1) / rows_per_cta);
     switch (vpt) {
-    case 1: launch_one<TEAM, 1>(p, stream); break;
-    case 2: launch_one<TEAM, 2>(p, stream); break;
-    case 3: launch_one<TEAM, 3>(p, stream); break;
-    case 4: launch_one<TEAM, 4>(p, stream); break;
-    case 5: launch_one<TEAM, 5>(p, stream); break;
-    case 6: launch_one<TEAM, 6>(p, stream); break;
-    case 7: launch_one<TEAM, 7>(p, stream); break;
-    case 8: launch_one<TEAM, 8>(p, stream); break;
-#if DIT_ADALN_MAX_VPT > 8
-    case 10: launch_one<TEAM, 10>(p, stream); break;
-    case 12: launch_one<TEAM, 12>(p, stream); break;
-    case 16: launch_one<TEAM, 16>(p, stream); break;
-    case 20: launch_one<TEAM, 20>(p, stream); break;
-    case 24: launch_one<TEAM, 24>(p, stream); break;
-#endif
+    case 4: adaln_team_kernel<4, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case 5: adaln_team_kernel<5, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case 6: adaln_team_kernel<6, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case 7: adaln_team_kernel<7, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case 8: adaln_team_kernel<8, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -343,42 +299,42 @@ cudaError_t launch_team(const AdalnParams& p, int vpt, cudaStream_t stream)
 
 }  // namespace
 
-// Team size: the smallest of 1, 2, 4, 8 warps that holds the row in at most
-// DIT_ADALN_MAX_VPT vectors per lane.
+// Rows of up to 6144 elements: one warp per row, VPT = ceil(hidden / 256)
+// vectors per lane rounded up to an instantiated count.  Wider rows (to
+// 16384): the smallest team of 2, 4 or 8 warps that holds the row in at most
+// 8 vectors per lane.
 cudaError_t launch_adaln_modulate(const AdalnParams& p, cudaStream_t stream)
 {
     const int nvec = p.hidden / 8;
-#if DIT_ADALN_PIPELINED
-    {
-#ifdef DIT_ADALN_STAGES
-        return launch_pipelined<DIT_ADALN_STAGES>(p, stream);
-#else
-        const int row_bytes = nvec * 16;
-        if (row_bytes <= 6 * 1024)
-            return launch_pipelined<8>(p, stream);
-        if (row_bytes <= 12 * 1024)
-            return launch_pipelined<4>(p, stream);
-        return launch_pipelined<2>(p, stream);
-#endif
-    }
-#endif
-    for (int team = 1; team <= kWarpsPerCta; team *= 2) {
-        const int per = team * kWarp;
-        int vpt = (nvec + per - 1) / per;
-        if (vpt > DIT_ADALN_MAX_VPT && team < kWarpsPerCta)
-            continue;
-        for (int s : kVptSteps)
-            if (s >= vpt && s <= DIT_ADALN_MAX_VPT) {
-                vpt = s;
-                break;
-            }
-        switch (team) {
-        case 1: return launch_team<1>(p, vpt, stream);
-        case 2: return launch_team<2>(p, vpt, stream);
-        case 4: return launch_team<4>(p, vpt, stream);
-        default: return launch_team<8>(p, vpt, stream);
+    const int vpt = (nvec + kWarp - 1) / kWarp;
+    if (vpt <= kMaxWarpVpt) {
+        switch (vpt) {
+        case 1: return launch_warp<1>(p, stream);
+        case 2: return launch_warp<2>(p, stream);
+        case 3: return launch_warp<3>(p, stream);
+        case 4: return launch_warp<4>(p, stream);
+        case 5: return launch_warp<5>(p, stream);
+        case 6: return launch_warp<6>(p, stream);
+        case 7: return launch_warp<7>(p, stream);
+        case 8: return launch_warp<8>(p, stream);
+        default: break;
         }
+        if (vpt <= 10)
+            return launch_warp<10>(p, stream);
+        if (vpt <= 12)
+            return launch_warp<12>(p, stream);
+        if (vpt <= 16)
+            return launch_warp<16>(p, stream);
+        if (vpt <= 20)
+            return launch_warp<20>(p, stream);
+        return launch_warp<24>(p, stream);
     }
+    if (nvec <= 2 * kWarp * 8)
+        return launch_team<2>(p, stream);
+    if (nvec <= 4 * kWarp * 8)
+        return launch_team<4>(p, stream);
+    if (nvec <= 8 * kWarp * 8)
+        return launch_team<8>(p, stream);
     return cudaErrorInvalidValue;  // hidden > kMaxAdalnHidden, rejected by the ABI first
 }
 

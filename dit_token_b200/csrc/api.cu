@@ -10,6 +10,10 @@
 #include "dit_token.h"
 #include "launch.h"
 
+static_assert(DIT_ROPE_INTERLEAVED == dit::kRopeInterleaved && DIT_ROPE_HALF == dit::kRopeHalf &&
+                  DIT_ROPE_NONE == dit::kRopeNone,
+              "rotary mode codes");
+
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
@@ -59,19 +63,37 @@ dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, int64_t k
                                const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
                                float rope_theta, float eps, void* stream)
 {
+    if (head_dim != 64 && head_dim != 128 && head_dim > 0)
+        return DIT_ERR_UNSUPPORTED;  // the original entry point keeps its documented range
+    return dit_qk_rmsnorm_rope_ex(q, q_row_stride, k, k_row_stride, q_weight, k_weight, cu_seqlens,
+                                  cu_seqlens_padded, num_seqs, num_rows_padded, num_q_heads, num_k_heads,
+                                  head_dim, rope_grid, sec_t, sec_h, sec_w, rope_theta, eps,
+                                  DIT_ROPE_INTERLEAVED, stream);
+}
+
+dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                                  const void* q_weight, const void* k_weight,
+                                  const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                  int32_t num_seqs, int64_t num_rows_padded,
+                                  int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+                                  const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+                                  float rope_theta, float eps, int32_t rope_mode, void* stream)
+{
     bool empty = false;
     dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
     if (st != DIT_OK)
         return st;
     if (num_q_heads < 0 || num_k_heads < 0 || head_dim <= 0)
         return DIT_ERR_SHAPE;
-    if (head_dim != 64 && head_dim != 128)
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+        return DIT_ERR_UNSUPPORTED;
+    if (rope_mode != DIT_ROPE_INTERLEAVED && rope_mode != DIT_ROPE_HALF && rope_mode != DIT_ROPE_NONE)
         return DIT_ERR_UNSUPPORTED;
     if (q_row_stride < (int64_t)num_q_heads * head_dim || k_row_stride < (int64_t)num_k_heads * head_dim)
         return DIT_ERR_SHAPE;
     if (!(rope_theta > 0.f) || !(eps >= 0.f) || !std::isfinite(rope_theta) || !std::isfinite(eps))
         return DIT_ERR_SHAPE;
-    if (rope_grid) {
+    if (rope_grid && rope_mode != DIT_ROPE_NONE) {
         if (sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t | sec_h | sec_w) & 1 ||
             (int64_t)sec_t + sec_h + sec_w != head_dim)
             return DIT_ERR_SHAPE;
@@ -90,7 +112,7 @@ dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, int64_t k
     p.k = static_cast<uint16_t*>(k);
     p.q_weight = static_cast<const uint16_t*>(q_weight);
     p.k_weight = static_cast<const uint16_t*>(k_weight);
-    p.rope_grid = rope_grid;
+    p.rope_grid = rope_mode == DIT_ROPE_NONE ? nullptr : rope_grid;
     p.q_row_stride = q_row_stride;
     p.k_row_stride = k_row_stride;
     p.pk = packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded);
@@ -114,9 +136,9 @@ dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, int64_t k
             first += sec[s] / 2;
         }
         p.axis[j] = (int8_t)axis;
-        p.inv_freq_3d[j] = rope_grid ? std::pow(theta, -2.0 * (j - first) / sec[axis]) : 0.0;
+        p.inv_freq_3d[j] = p.rope_grid ? std::pow(theta, -2.0 * (j - first) / sec[axis]) : 0.0;
     }
-    return from_cuda(dit::launch_qk_rmsnorm_rope(p, head_dim, static_cast<cudaStream_t>(stream)));
+    return from_cuda(dit::launch_qk_rmsnorm_rope(p, head_dim, rope_mode, static_cast<cudaStream_t>(stream)));
 }
 
 dit_status dit_adaln_modulate(const void* x, int64_t x_row_stride, void* out, int64_t out_row_stride,

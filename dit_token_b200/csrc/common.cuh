@@ -74,6 +74,40 @@ __device__ __forceinline__ bool map_valid_row(int v, const int32_t* __restrict__
     return true;
 }
 
+// Walks valid-row ordinals upward for a persistent CTA that owns a contiguous
+// range of them: the padded row of the next ordinal is the previous one + 1
+// except at a sequence boundary, so global loads happen only when a boundary
+// is crossed.  Every thread of the CTA holds the same state.
+struct RowCursor {
+    const int32_t* cs;
+    const int32_t* cp;
+    int B;
+    int rows_padded;
+    int b;  // current sequence
+    int cs0, cs1, cp0, cp1;
+
+    __device__ __forceinline__ void load(int bb)
+    {
+        b = bb;
+        cs0 = __ldg(cs + b);
+        cs1 = __ldg(cs + b + 1);
+        cp0 = __ldg(cp + b);
+        cp1 = __ldg(cp + b + 1);
+    }
+    // Padded row of ordinal v (v never decreases between calls), or -1 when v
+    // is not a valid row or the descriptor points outside the buffer.
+    __device__ __forceinline__ int row(int v)
+    {
+        while (v >= cs1 && b + 1 < B)
+            load(b + 1);
+        const int r = v - cs0;
+        if (r < 0 || r >= cs1 - cs0 || r >= cp1 - cp0)
+            return -1;
+        const long long rr = (long long)cp0 + r;
+        return rr < rows_padded ? (int)rr : -1;
+    }
+};
+
 // ---------------------------------------------------------- vector I/O
 // Streamed activations are touched once: load and store them with the
 // evict-first (".cs") policy so they do not push the small per-sequence
@@ -125,19 +159,38 @@ __device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
     f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
 }
 
-// The same widening as an opaque instruction, so that a later pass over
-// register-resident packed data recomputes it instead of keeping eight fp32
-// copies per vector alive (which would cost occupancy in the row kernels).
-__device__ __forceinline__ void unpack8_again(uint4 v, float (&f)[8])
+// ------------------------------------------------ packed fp32 pairs
+// sm_100 executes add/mul/fma on two fp32 lanes of a 64-bit register pair in
+// one instruction (PTX .f32x2); the row kernels that are bound by instruction
+// issue rather than by HBM use these for their element-wise arithmetic.
+// The pairs are float2 values operated on with the sm_100 packed builtins
+// (__fadd2_rn, __ffma2_rn ...), so the compiler allocates register pairs itself.
+typedef float2 f32x2;
+
+__device__ __forceinline__ f32x2 f2_make(float lo, float hi) { return make_float2(lo, hi); }
+
+__device__ __forceinline__ void f2_split(f32x2 v, float& lo, float& hi)
 {
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t lo, hi;
-        asm volatile("shl.b32 %0, %2, 16;\n\tand.b32 %1, %2, 0xffff0000;" : "=r"(lo), "=r"(hi) : "r"(w[i]));
-        f[2 * i] = __uint_as_float(lo);
-        f[2 * i + 1] = __uint_as_float(hi);
-    }
+    lo = v.x;
+    hi = v.y;
+}
+
+// bf16x2 word (element 0 in the low half) -> the two values as an fp32 pair.
+__device__ __forceinline__ f32x2 f2_from_bf16x2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) { return __ffma2_rn(a, b, c); }
+
+// fp32 pair -> bf16x2 word, round to nearest even.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(f32x2 v)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
+    return r;
 }
 
 // Two fp32 values -> one bf16x2 word (round to nearest, ties to even).
@@ -174,6 +227,48 @@ struct MinCtas {
     static constexpr int raw = 65536 / (kCtaThreads * regs);
     static constexpr int value = raw < 1 ? 1 : (raw > 8 ? 8 : raw);
 };
+
+// ----------------------------------------------- row mean / variance
+// LayerNorm statistics in one pass, robust to large means and outliers: each
+// thread accumulates s = sum(x - k) and q = sum((x - k)^2) about its own first
+// value k, turns them into (count, mean, M2 = sum of squared deviations), and
+// the partial moments are merged pairwise (Chan, Golub and LeVeque's update):
+//   n = na + nb,  d = mb - ma,  mean = ma + d nb / n,  M2 = Ma + Mb + d^2 na nb / n.
+// The merge order is fixed, so the result is bitwise reproducible.
+struct Moments {
+    float n, mean, m2;
+};
+
+__device__ __forceinline__ Moments moments_merge(Moments a, Moments b)
+{
+    const float n = a.n + b.n;
+    if (n == 0.f)
+        return a;
+    const float d = b.mean - a.mean;
+    const float wb = __fdividef(b.n, n);  // a weight in [0, 1]: the fast quotient is ample
+    return Moments{n, fmaf(d, wb, a.mean), a.m2 + b.m2 + d * d * a.n * wb};
+}
+
+__device__ __forceinline__ Moments moments_from_sums(float n, float k, float s, float q)
+{
+    if (n == 0.f)
+        return Moments{0.f, 0.f, 0.f};
+    const float m = __fdividef(s, n);
+    return Moments{n, k + m, fmaxf(q - s * m, 0.f)};
+}
+
+// Merge over the 32 lanes of a warp (xor butterfly: every lane ends with the total).
+__device__ __forceinline__ Moments moments_warp(Moments m)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        Moments other{__shfl_xor_sync(0xffffffffu, m.n, o), __shfl_xor_sync(0xffffffffu, m.mean, o),
+                      __shfl_xor_sync(0xffffffffu, m.m2, o)};
+        // lanes of a pair merge in the same (lower lane first) order
+        m = (threadIdx.x & o) ? moments_merge(other, m) : moments_merge(m, other);
+    }
+    return m;
+}
 
 template <int WIDTH>
 __device__ __forceinline__ float group_sum(float v)

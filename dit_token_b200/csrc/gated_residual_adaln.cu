@@ -5,13 +5,15 @@
 // "Why Real-Time MiniMax H3 Serving Requires More Than a Faster DiT", "Key
 // takeaways", bullet 2 lists residual updates next to modulation and
 // normalization among the fused work.  LN reads the residual as stored
-// (rounded to bf16), so the pair equals the two separate ops back to back,
-// bit for bit up to the fp32 reduction order -- while HBM sees x and y read
-// once and res and norm written once: 8 bytes per element instead of the
-// 10 of the unfused pair.
+// (rounded to bf16), so the pair equals the two separate ops back to back
+// (the residual bit for bit; the normalization up to the order in which the
+// row statistics are merged) -- while HBM sees x and y read once and res and
+// norm written once: 8 bytes per element instead of the 10 of the unfused
+// pair.
 //
 // Layout as in adaln_modulate.cu: a team of TEAM warps owns a row and keeps
-// the rounded residual in registers (VPT 16-byte vectors per lane).
+// the rounded residual in registers (VPT 16-byte vectors per lane); one-pass
+// moments for the statistics, packed fp32 pairs for the arithmetic.
 #include "common.cuh"
 #include "launch.h"
 
@@ -24,7 +26,7 @@ gated_residual_adaln_kernel(const FusedParams p)
 {
     constexpr int kRowsPerCta = kWarpsPerCta / TEAM;
     constexpr int kTeamThreads = TEAM * kWarp;
-    __shared__ float red[2][kWarpsPerCta];
+    __shared__ Moments red[kWarpsPerCta];
 
     const int lane = threadIdx.x & (kWarp - 1);
     const int warp = threadIdx.x >> 5;
@@ -57,14 +59,15 @@ gated_residual_adaln_kernel(const FusedParams p)
         for (int i = 0; i < VPT; ++i) {
             const int j = i * kTeamThreads + tt;
             if (j < nvec) {
-                float xf[8], yf[8], gf[8], o[8];
-                unpack8(xv[i], xf);
-                unpack8(yv[i], yf);
-                unpack8(ld_shared_vec(gr + 8 * j), gf);
+                const uint4 gv = ld_shared_vec(gr + 8 * j);
+                const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+                const uint32_t yw[4] = {yv[i].x, yv[i].y, yv[i].z, yv[i].w};
+                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                uint32_t o[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    o[e] = fmaf(gf[e], yf[e], xf[e]);
-                rv[i] = pack8(o);
+                for (int e = 0; e < 4; ++e)
+                    o[e] = f2_to_bf16x2(f2_fma(f2_from_bf16x2(gw[e]), f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
+                rv[i] = make_uint4(o[0], o[1], o[2], o[3]);
                 st_stream(res + 8 * j, rv[i]);
             } else {
                 rv[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -72,53 +75,43 @@ gated_residual_adaln_kernel(const FusedParams p)
         }
     }
 
-    // LN statistics of the stored residual
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        float f[8];
-        unpack8(rv[i], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            sum += f[e];
-    }
-    sum = group_sum<kWarp>(sum);
-    if (TEAM > 1) {
-        if (lane == 0)
-            red[0][warp] = sum;
-        team_barrier<TEAM>(team);
-        sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < TEAM; ++w)
-            sum += red[0][team * TEAM + w];
-    }
-    const float inv_n = 1.0f / (float)p.hidden;
-    const float mean = sum * inv_n;
-    float sq = 0.f;
+    // LN statistics of the stored residual: shifted sums, merged as moments
+    const float k = bf16_lo(rv[0].x);
+    const f32x2 kk = f2_make(k, k);
+    f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
+    float cnt = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
-            float f[8];
-            unpack8_again(rv[i], f);
+            const uint32_t w[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = f[e] - mean;
-                sq = fmaf(d, d, sq);
+            for (int e = 0; e < 4; ++e) {
+                const f32x2 d = f2_sub(f2_from_bf16x2(w[e]), kk);
+                s2 = f2_add(s2, d);
+                q2 = f2_fma(d, d, q2);
             }
+            cnt += 8.f;
         }
     }
-    sq = group_sum<kWarp>(sq);
+    float s0, s1, q0, q1;
+    f2_split(s2, s0, s1);
+    f2_split(q2, q0, q1);
+    Moments m = moments_warp(moments_from_sums(cnt, k, s0 + s1, q0 + q1));
     if (TEAM > 1) {
         if (lane == 0)
-            red[1][warp] = sq;
+            red[warp] = m;
         team_barrier<TEAM>(team);
-        sq = 0.f;
+        m = red[team * TEAM];
 #pragma unroll
-        for (int w = 0; w < TEAM; ++w)
-            sq += red[1][team * TEAM + w];
+        for (int w = 1; w < TEAM; ++w)
+            m = moments_merge(m, red[team * TEAM + w]);
     }
-    const float rstd = rsqrtf(sq * inv_n + p.eps);
+    const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);  // as in adaln_modulate.cu
+    const f32x2 r2 = f2_make(rstd, rstd);
+    const float nb = -m.mean * rstd;
+    const f32x2 b2 = f2_make(nb, nb);
+    const f32x2 one2 = f2_make(1.f, 1.f);
 
     const uint16_t* sh = p.shift + (int64_t)s.seq * p.mod_seq_stride;
     const uint16_t* sc = p.scale + (int64_t)s.seq * p.mod_seq_stride;
@@ -127,14 +120,18 @@ gated_residual_adaln_kernel(const FusedParams p)
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
-            float f[8], shf[8], scf[8], o[8];
-            unpack8_again(rv[i], f);
-            unpack8(ld_shared_vec(sh + 8 * j), shf);
-            unpack8(ld_shared_vec(sc + 8 * j), scf);
+            const uint4 shv = ld_shared_vec(sh + 8 * j);
+            const uint4 scv = ld_shared_vec(sc + 8 * j);
+            const uint32_t rw[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
+            const uint32_t hw[4] = {shv.x, shv.y, shv.z, shv.w};
+            const uint32_t cw[4] = {scv.x, scv.y, scv.z, scv.w};
+            uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                o[e] = fmaf((f[e] - mean) * rstd, 1.0f + scf[e], shf[e]);
-            st_stream(nrow + 8 * j, pack8(o));
+            for (int e = 0; e < 4; ++e) {
+                const f32x2 t = f2_fma(f2_from_bf16x2(rw[e]), r2, b2);
+                o[e] = f2_to_bf16x2(f2_fma(t, f2_add(f2_from_bf16x2(cw[e]), one2), f2_from_bf16x2(hw[e])));
+            }
+            st_stream(nrow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
         }
     }
 }

@@ -15,7 +15,12 @@ struct Packing {
     int32_t num_rows_padded;
 };
 
-constexpr int kMaxPairs = 64;  // head_dim <= 128
+constexpr int kMaxPairs = 128;  // head_dim <= 256
+
+// Rotary layouts of dit_qk_rmsnorm_rope_ex (the DIT_ROPE_* values of the ABI).
+constexpr int kRopeInterleaved = 0;
+constexpr int kRopeHalf = 1;
+constexpr int kRopeNone = 2;
 
 struct QkParams {
     uint16_t* q;
@@ -101,7 +106,7 @@ struct FramesParams {
 };
 
 cudaError_t launch_frames_to_u8(const FramesParams& p, cudaStream_t stream);
-cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, cudaStream_t stream);
+cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, int rope_mode, cudaStream_t stream);
 cudaError_t launch_adaln_modulate(const AdalnParams& p, cudaStream_t stream);
 cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream);
 cudaError_t launch_swiglu(const SwigluParams& p, cudaStream_t stream);

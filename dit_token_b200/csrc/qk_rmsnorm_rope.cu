@@ -4,15 +4,14 @@
 // takeaways", bullet 2: the Q/K normalization is fused with the rotary
 // embedding; bullet 1: rotary rows are computed only where needed).
 //
-// Layout.  One warp per valid row.  A head of D = 8*LPH elements is held by a
-// group of LPH lanes, 8 elements (one 16-byte vector) per lane, so the
-// per-head sum of squares is a log2(LPH)-step xor-shuffle reduction and every
-// lane owns 4 complete interleaved pairs (2j, 2j+1): the rotation is
-// lane-local.  A lane always sits at the same offset inside a head, so it
-// needs the cos/sin of only its own 4 pairs: it computes them once per row
-// (angle reduced in fp64, then sincosf) and reuses them for all
-// num_q_heads + num_k_heads heads of that row -- cos/sin are never re-read or
-// recomputed per head.  Each step issues U head vectors per lane before any
+// Layout.  One warp per valid row.  A head of D = 8*LPH elements (D = 64,
+// 128 or 256) is held by a group of LPH lanes, 8 elements (one 16-byte vector)
+// per lane, so the per-head sum of squares is a log2(LPH)-step xor-shuffle
+// reduction.  A lane always sits at the same offset inside a head, so it
+// needs the cos/sin of only its own pairs (4 interleaved, 8 half-split): it
+// computes them once per row (angle reduced in fp64, then sincosf) and reuses
+// them for all num_q_heads + num_k_heads heads of that row -- cos/sin are
+// never re-read or recomputed per head.  Each step issues U head vectors per lane before any
 // arithmetic.  HBM traffic: q and k are each read once and written once, 4
 // bytes per element.
 #include "common.cuh"
@@ -36,12 +35,18 @@ __device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
     sincosf((float)red, &s, &c);
 }
 
-template <int D>
+// Rotary layouts (template MODE): pair j of a head is (2j, 2j+1) when
+// interleaved -- all four of a lane's pairs are inside its own 8 elements --
+// or (j, j + D/2) when half-split -- a lane then holds one side of 8 pairs and
+// the lane LPH/2 away holds the other side, fetched with one xor shuffle per
+// element.  MODE none applies the RMSNorm and the weight only.
+template <int D, int MODE>
 __global__ void __launch_bounds__(kCtaThreads)
 qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
 {
     constexpr int LPH = D / 8;          // lanes per head
     constexpr int HPW = kWarp / LPH;    // heads per warp per step
+    constexpr int NP = MODE == kRopeHalf ? 8 : (MODE == kRopeInterleaved ? 4 : 0);  // pairs per lane
     const int lane = threadIdx.x & (kWarp - 1);
     const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     RowSlot s;
@@ -50,35 +55,38 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         return;
     const int sub = lane / LPH;  // which head of the step
     const int li = lane % LPH;   // position inside the head: elements 8*li .. 8*li+7
+    const bool upper = MODE == kRopeHalf && li >= LPH / 2;  // holds the j + D/2 side
 
-    // Positions of this row: a row inside the sequence's T x H x W video grid
-    // (t-major, then h, then w) is 3D; every later row is 1D, counted from the
-    // end of the grid.  Without a grid every row is 1D.
-    bool is3d = false;
-    long long pt = 0, ph = 0, pw = 0;
-    long long pos1 = s.local;
-    if (p.rope_grid != nullptr) {
-        const long long T = __ldg(p.rope_grid + 3 * s.seq);
-        const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
-        const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
-        const long long thw = T * H * W;
-        if (s.local < thw) {
-            is3d = true;
-            pt = s.local / (H * W);
-            ph = (s.local / W) % H;
-            pw = s.local % W;
-        } else {
-            pos1 = s.local - thw;
+    float cs[NP > 0 ? NP : 1], sn[NP > 0 ? NP : 1];
+    if (NP > 0) {
+        // Positions of this row: a row inside the sequence's T x H x W video
+        // grid (t-major, then h, then w) is 3D; every later row is 1D, counted
+        // from the end of the grid.  Without a grid every row is 1D.
+        bool is3d = false;
+        long long pt = 0, ph = 0, pw = 0;
+        long long pos1 = s.local;
+        if (p.rope_grid != nullptr) {
+            const long long T = __ldg(p.rope_grid + 3 * s.seq);
+            const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
+            const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
+            const long long thw = T * H * W;
+            if (s.local < thw) {
+                is3d = true;
+                pt = s.local / (H * W);
+                ph = (s.local / W) % H;
+                pw = s.local % W;
+            } else {
+                pos1 = s.local - thw;
+            }
         }
-    }
-    float cs[4], sn[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int j = 4 * li + e;
-        const int ax = p.axis[j];
-        const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
-        const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
-        pair_cos_sin(ang, cs[e], sn[e]);
+        for (int e = 0; e < NP; ++e) {
+            const int j = MODE == kRopeHalf ? 8 * (li % (LPH / 2)) + e : 4 * li + e;
+            const int ax = p.axis[j];
+            const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
+            const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
+            pair_cos_sin(ang, cs[e], sn[e]);
+        }
     }
     float wq[8], wk[8];
     unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
@@ -110,35 +118,58 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
             for (int e = 0; e < 8; ++e)
                 ss = fmaf(x[e], x[e], ss);
             ss = group_sum<LPH>(ss);  // every lane of the warp takes part
-            if (h < Htot) {
-                const float r = rsqrtf(ss * inv_d + p.eps);
-                const bool isq = h < Hq;
-                float o[8];
+            const float r = rsqrtf(ss * inv_d + p.eps);
+            const bool isq = h < Hq;
+            float y[8], o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                y[e] = x[e] * r * (isq ? wq[e] : wk[e]);
+            if (MODE == kRopeInterleaved) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float y0 = x[2 * e] * r * (isq ? wq[2 * e] : wk[2 * e]);
-                    const float y1 = x[2 * e + 1] * r * (isq ? wq[2 * e + 1] : wk[2 * e + 1]);
-                    o[2 * e] = y0 * cs[e] - y1 * sn[e];
-                    o[2 * e + 1] = y0 * sn[e] + y1 * cs[e];
+                    o[2 * e] = y[2 * e] * cs[e] - y[2 * e + 1] * sn[e];
+                    o[2 * e + 1] = y[2 * e] * sn[e] + y[2 * e + 1] * cs[e];
                 }
-                st_stream(isq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D, pack8(o));
+            } else if (MODE == kRopeHalf) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float partner = __shfl_xor_sync(0xffffffffu, y[e], LPH / 2);  // all lanes take part
+                    o[e] = upper ? partner * sn[e] + y[e] * cs[e] : y[e] * cs[e] - partner * sn[e];
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    o[e] = y[e];
             }
+            if (h < Htot)
+                st_stream(isq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D, pack8(o));
         }
     }
 }
 
+template <int D>
+cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
+{
+    switch (mode) {
+    case kRopeInterleaved: qk_rmsnorm_rope_kernel<D, kRopeInterleaved><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeHalf: qk_rmsnorm_rope_kernel<D, kRopeHalf><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeNone: qk_rmsnorm_rope_kernel<D, kRopeNone><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, cudaStream_t stream)
+cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, int rope_mode, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)((p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta);
-    if (head_dim == 128)
-        qk_rmsnorm_rope_kernel<128><<<grid, kCtaThreads, 0, stream>>>(p);
-    else if (head_dim == 64)
-        qk_rmsnorm_rope_kernel<64><<<grid, kCtaThreads, 0, stream>>>(p);
-    else
-        return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    switch (head_dim) {
+    case 64: return launch_d<64>(p, rope_mode, grid, stream);
+    case 128: return launch_d<128>(p, rope_mode, grid, stream);
+    case 256: return launch_d<256>(p, rope_mode, grid, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace dit

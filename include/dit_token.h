@@ -105,6 +105,29 @@ DIT_API dit_status dit_qk_rmsnorm_rope(void* q, int64_t q_row_stride, void* k, i
                                const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
                                float rope_theta, float eps, void* stream);
 
+/* dit_qk_rmsnorm_rope with a choice of rotary layout and head_dim 64, 128 or
+ * 256.  No counterpart on the pages beyond the operator itself: they do not
+ * say how Q/K are laid out, so the layout is a parameter.
+ *   DIT_ROPE_INTERLEAVED  pairs (2j, 2j+1)       -- what dit_qk_rmsnorm_rope does
+ *   DIT_ROPE_HALF         pairs (j, j + D/2)     ("rotate half" layout); same angles
+ *   DIT_ROPE_NONE         per-head RMSNorm times the weight, no rotation (rope_grid
+ *                         and sections are ignored) -- the Q/K normalization of
+ *                         attention blocks without positional rotation, e.g. the
+ *                         VAE's (third page, "vLLM-Omni 中的系统级优化", bullet 3)
+ * Every other argument is as for dit_qk_rmsnorm_rope; an unknown mode or a
+ * head_dim outside {64, 128, 256} returns DIT_ERR_UNSUPPORTED. */
+#define DIT_ROPE_INTERLEAVED 0
+#define DIT_ROPE_HALF 1
+#define DIT_ROPE_NONE 2
+DIT_API dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                                          const void* q_weight, const void* k_weight,
+                                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                          int32_t num_seqs, int64_t num_rows_padded,
+                                          int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+                                          const int32_t* rope_grid, int32_t sec_t, int32_t sec_h,
+                                          int32_t sec_w, float rope_theta, float eps, int32_t rope_mode,
+                                          void* stream);
+
 /* Adaptive LayerNorm modulation: out = LN(x) * (1 + scale_b) + shift_b.
  *
  * Pages: first page "Key takeaways" bullet 2 (the modulation and the

@@ -53,14 +53,14 @@ def device_packing(w: W.Workload):
 
 # ------------------------------------------------------------ GPU runs
 
-def gpu_qk(w, inp, dev=None):
+def gpu_qk(w, inp, rope_mode="interleaved"):
     cs, cp, grid = device_packing(w)
     q = inp["q"].cuda()
     k = inp["k"].cuda()
     dit.dit_qk_rmsnorm_rope(W.rows_view(q), W.rows_view(k), inp["q_weight"].cuda(), inp["k_weight"].cuda(),
                             cs, cp, num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads,
                             head_dim=w.head_dim, rope_grid=grid, sections=w.sections,
-                            rope_theta=w.rope_theta, eps=w.eps)
+                            rope_theta=w.rope_theta, eps=w.eps, rope_mode=rope_mode)
     return q, k
 
 
@@ -107,13 +107,14 @@ def gpu_swiglu(w, inp):
 
 # ------------------------------------------------------------ oracle runs
 
-def oracle_qk(w, inp, rows):
+def oracle_qk(w, inp, rows, rope_mode="interleaved"):
     q = tbits(W.rows_view(inp["q"]))
     k = tbits(W.rows_view(inp["k"]))
     return oracle.qk_rmsnorm_rope(q, k, tbits(inp["q_weight"]), tbits(inp["k_weight"]), w.cu_seqlens,
                                   w.cu_seqlens_padded, num_q_heads=w.num_q_heads,
                                   num_k_heads=w.num_k_heads, head_dim=w.head_dim, rope_grid=w.rope_grid,
-                                  sections=w.sections, rope_theta=w.rope_theta, eps=w.eps, rows=rows)
+                                  sections=w.sections, rope_theta=w.rope_theta, eps=w.eps, rows=rows,
+                                  rope_mode=rope_mode)
 
 
 def oracle_adaln(w, inp, rows):

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 10, names
+    assert len(names) == 11, names
     for n in names:
         assert hasattr(L, n), n
     assert L.dit_abi_version() == 1
@@ -69,6 +69,20 @@ def test_qk_argument_checks(L):
     assert qk(L, theta=0.0) == SHAPE
     assert qk(L, eps=float("nan")) == SHAPE
     assert qk(L, grid=P + 2, st=44, sh=42, sw=42) == ALIGN
+
+
+def test_qk_ex_argument_checks(L):
+    def ex(mode, d=128, **kw):
+        a = dict(q=P, qs=512, k=P, ks=512, grid=None, st=0, sh=0, sw=0)
+        a.update(kw)
+        return L.dit_qk_rmsnorm_rope_ex(a["q"], a["qs"], a["k"], a["ks"], P, P, P, P, 1, 16, 2, 2, d, a["grid"],
+                                        a["st"], a["sh"], a["sw"], 10000.0, 1e-6, mode, None)
+    assert ex(3) == UNSUP and ex(-1) == UNSUP
+    assert ex(0, d=512, qs=1024, ks=1024) == UNSUP
+    assert ex(1, d=256, qs=500) == SHAPE
+    assert ex(1, grid=P, st=44, sh=42, sw=40) == SHAPE
+    assert ex(2, grid=P, st=44, sh=42, sw=40, q=None) == NULL   # sections are ignored without rotation
+    assert qk(L, d=256, qs=512, ks=512) == UNSUP                # the original entry keeps 64/128
 
 
 def test_empty_batches_launch_nothing(L):

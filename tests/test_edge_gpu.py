@@ -76,6 +76,31 @@ def test_head_dim_64_with_3d_sections_and_gqa():
     all_ops_full(ragged(head_dim=64, sections=(24, 20, 20), hq=4, hk=2, hidden=264, inner=520))
 
 
+@pytest.mark.parametrize("mode", ["interleaved", "half", "none"])
+@pytest.mark.parametrize("head_dim,sections", [(64, (24, 20, 20)), (128, (44, 42, 42)), (256, (88, 84, 84))])
+def test_rope_modes_and_head_dims(mode, head_dim, sections):
+    w = ragged(head_dim=head_dim, sections=sections, hq=3, hk=2, hidden=264, inner=264, seed=head_dim)
+    rows = w.valid_rows()
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp, rope_mode=mode)
+    qo, ko = P.oracle_qk(w, inp, rows, rope_mode=mode)
+    P.assert_close(P.gather_rows(q, rows), qo[rows], f"q {mode} {head_dim}")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], f"k {mode} {head_dim}")
+    keep = P.untouched_rows(w)
+    P.assert_untouched(q, inp["q"], keep, "q")
+    P.assert_untouched(k, inp["k"], keep, "k")
+
+
+def test_half_split_video_full_size_sampled():
+    w = W.workload("video")
+    rows = W.sample_rows(w, per_seq=64)
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp, rope_mode="half")
+    qo, ko = P.oracle_qk(w, inp, rows, rope_mode="half")
+    P.assert_close(P.gather_rows(q, rows), qo[rows], "q half video")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], "k half video")
+
+
 def test_1d_only_and_degenerate_sections():
     w = W.custom("1d", (77, 3), (80, 8), hidden=512, num_q_heads=2, num_k_heads=2, head_dim=128, inner=256)
     all_ops_full(w)

@@ -88,7 +88,9 @@ def test_gated_residual_adaln(case):
     keep = P.untouched_rows(w)
     P.assert_untouched(res, inp["out"], keep, f"{w.name} fused res")
     P.assert_untouched(norm, inp["out"], keep, f"{w.name} fused norm")
-    # the fused op reproduces the two separate kernels bit for bit
+    # the fused op's residual is the separate kernel's bit for bit; its
+    # normalization agrees with the separate adaLN kernel (whose statistics are
+    # merged in another order) within the same tolerance
     import dit_token_b200 as dit
     cs, cp, _ = P.device_packing(w)
     mod = inp["mod"].cuda()
@@ -96,4 +98,4 @@ def test_gated_residual_adaln(case):
     n2 = W.sentinel_like(inp["out"].shape).cuda()
     dit.dit_adaln_modulate(W.rows_view(r2), mod[:, 3], mod[:, 4], cs, cp, out=W.rows_view(n2), eps=w.eps)
     assert torch.equal(res.view(torch.int16), r2.view(torch.int16))
-    assert torch.equal(norm.view(torch.int16), n2.view(torch.int16))
+    P.assert_close(P.gather_rows(norm, rows), P.gather_rows(n2, rows), f"{w.name} fused vs separate adaLN")
