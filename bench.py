@@ -31,6 +31,7 @@ import argparse
 import dataclasses
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -52,6 +53,7 @@ METRIC = "fused DiT token-op throughput (tokens/s, achieved HBM GB/s, % of roofl
 UNIT = "tokens/s"
 OPS = ("qk_rmsnorm_rope", "adaln_modulate", "gated_residual", "swiglu")
 FALLBACK_HBM_GBS = 6650.0
+FRAMES_ELEMS = 1 * 3 * 243 * 768 * 1344
 PROFILES = os.path.join(ROOT, "profiles")
 
 
@@ -247,7 +249,14 @@ class Step:
                 events[op][1].record()
 
 
-def time_next_ops(step: Step, steps: int, warmup: int, device) -> dict:
+def frames_shape(scale: float = 1.0):
+    """Decoded-frame tensor of the pages' request, its frame count scaled with
+    the workload."""
+    B, C, T, H, Wd = W.FRAMES_SHAPE
+    return (B, C, max(1, int(round(T * scale))), H, Wd)
+
+
+def time_next_ops(step: Step, steps: int, warmup: int, device, scale: float = 1.0) -> dict:
     """Mean launch time of the operators built beyond the four-op step (same
     buffers, same stream), each timed on its own."""
     w, d, rv = step.w, step.dit, W.rows_view
@@ -256,8 +265,15 @@ def time_next_ops(step: Step, steps: int, warmup: int, device) -> dict:
         d.dit_gated_residual_adaln(rv(step.rx), rv(step.ry), step.mod[:, 2], step.mod[:, 3], step.mod[:, 4],
                                    step.cs, step.cp, res_out=rv(step.rout), norm_out=rv(step.aout), eps=w.eps)
 
+    fshape = frames_shape(scale)
+    frames_in = W.frames_input(fshape, seed=step.w.seed).to(step.q.device)
+    frames_out = torch.empty(fshape[0:1] + fshape[2:] + fshape[1:2], dtype=torch.uint8, device=step.q.device)
+
+    def frames():
+        d.dit_frames_to_u8(frames_in, layout="bthwc", out=frames_out)
+
     out = {}
-    for name, fn in (("gated_residual_adaln", fused),):
+    for name, fn in (("gated_residual_adaln", fused), ("frames_to_u8", frames)):
         for _ in range(warmup):
             fn()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -318,14 +334,15 @@ def time_e2e(sets, steps: int, warmup: int, device):
     h2d = sum(h.numel() * h.element_size() for op in OPS for h in h_in[op])
     d2h = sum(h.numel() * h.element_size() for op in OPS for h in h_out[op])
     s_up, s_run, s_down = (torch.cuda.Stream(device) for _ in range(3))
-    free = [None, None]
+    free = [None] * len(sets)
 
     def one(k):
-        st = sets[k % 2]
+        slot = k % len(sets)
+        st = sets[slot]
         ready, done = {}, {}
         with torch.cuda.stream(s_up):
-            if free[k % 2] is not None:
-                s_up.wait_event(free[k % 2])
+            if free[slot] is not None:
+                s_up.wait_event(free[slot])
             for op in OPS:
                 for d, h in zip(st.op_inputs(op), h_in[op]):
                     d.copy_(h, non_blocking=True)
@@ -342,8 +359,8 @@ def time_e2e(sets, steps: int, warmup: int, device):
                 s_down.wait_event(done[op])
                 for h, d in zip(h_out[op], st.op_outputs(op)):
                     h.copy_(d, non_blocking=True)
-            free[k % 2] = torch.cuda.Event()
-            free[k % 2].record(s_down)
+            free[slot] = torch.cuda.Event()
+            free[slot].record(s_down)
 
     for k in range(warmup):
         one(k)
@@ -466,9 +483,14 @@ def run_dit(args):
     clocks = sampler.summary(h0, h1)
     max_ms = reduce_max(elapsed_ms, device)
     op_ms_max = {op: reduce_max(v, device) for op, v in op_ms.items()}
-    next_ms = {k: reduce_max(v, device) for k, v in time_next_ops(step, args.steps, args.warmup, device).items()}
+    next_ms = {k: reduce_max(v, device)
+               for k, v in time_next_ops(step, args.steps, args.warmup, device, args.scale).items()}
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    e2e_ms, h2d, d2h = time_e2e([step, Step(w, host, device)], e2e_steps, min(args.warmup, 3), device)
+    # two device buffer sets let consecutive end-to-end steps overlap; one step needs one
+    # two device buffer sets let consecutive end-to-end steps overlap; the
+    # small profiling-size runs (--scale < 1) keep one to stay small
+    sets = [step, Step(w, host, device)] if args.scale >= 1.0 else [step]
+    e2e_ms, h2d, d2h = time_e2e(sets, e2e_steps, min(args.warmup, 3), device)
     e2e_max = reduce_max(e2e_ms, device)
 
     tokens = w.num_valid * world
@@ -502,6 +524,12 @@ def run_dit(args):
                 "gbs": round(8 * w.hidden * w.num_valid / (next_ms["gated_residual_adaln"] / 1e3) / 1e9, 1),
                 "bytes": 8 * w.hidden * w.num_valid,
                 "unfused_us": round((op_ms_max["gated_residual"] + op_ms_max["adaln_modulate"]) * 1e3, 2)},
+            "frames_to_u8": {
+                "workload": f"fp32 {list(frames_shape(args.scale))} -> uint8 BTHWC (the pages' 10 s 1344x768 "
+                            "request: 243 frames)",
+                "us": round(next_ms["frames_to_u8"] * 1e3, 2),
+                "gbs": round(5 * math.prod(frames_shape(args.scale)) / (next_ms["frames_to_u8"] / 1e3) / 1e9, 1),
+                "bytes": 5 * math.prod(frames_shape(args.scale))},
         },
         "e2e": {"value": round(tokens * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -547,31 +575,58 @@ def run_reference(args):
 
 
 def run_table(args):
-    """Per-op table over every workload (markdown on stdout): the measured
-    results that complement the single JSON line."""
+    """Per-op table over every workload (markdown on stdout), complementing the
+    single JSON line.  Each launch is preceded by a 512 MB write that evicts
+    L2 (the small workloads would otherwise be served from L2) and keeps the
+    GPU busy while the next launch is submitted, so the CUDA events around the
+    launch see the kernel alone."""
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     from dit_token_b200 import build
     build.build()
+    import dit_token_b200 as dit
     peak, kind = measured_peak()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.fill_(1)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(device)
+        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3  # us
+
     print(f"| workload | op | GPU us | tokens/s | GB/s | % of 8 TB/s | % of {kind} {peak:.0f} GB/s |")
     print("|---|---|---|---|---|---|---|")
     for name in W.WORKLOAD_NAMES:
         w = W.workload(name, args.seed)
         host = host_inputs(w)
         step = Step(w, host, device)
-        _, op_ms, _ = time_device(step, args.steps, args.warmup, device)
-        nxt = time_next_ops(step, args.steps, args.warmup, device)
+        rv = W.rows_view
         ab = algorithmic_bytes(w)
         ab["gated_residual_adaln"] = 8 * w.hidden * w.num_valid
-        op_ms.update(nxt)
-        for op in list(OPS) + ["gated_residual_adaln"]:
-            us = op_ms[op] * 1e3
+        fns = {op: (lambda op=op: step.run_op(op)) for op in OPS}
+        fns["gated_residual_adaln"] = lambda: dit.dit_gated_residual_adaln(
+            rv(step.rx), rv(step.ry), step.mod[:, 2], step.mod[:, 3], step.mod[:, 4], step.cs, step.cp,
+            res_out=rv(step.rout), norm_out=rv(step.aout), eps=w.eps)
+        for op, fn in fns.items():
+            us = timed(fn)
             gbs = ab[op] / (us * 1e-6) / 1e9
             print(f"| {name} | {op} | {us:.1f} | {w.num_valid / (us * 1e-6):.3g} | {gbs:.0f} | "
                   f"{100 * gbs / 8000:.1f} | {100 * gbs / peak:.1f} |", flush=True)
-        del step, host
+        del step, host, fns
         torch.cuda.empty_cache()
+    fin = W.frames_input(W.FRAMES_SHAPE, seed=args.seed).to(device)
+    fout = torch.empty((1, 243, 768, 1344, 3), dtype=torch.uint8, device=device)
+    us = timed(lambda: dit.dit_frames_to_u8(fin, layout="bthwc", out=fout))
+    gbs = 5 * FRAMES_ELEMS / (us * 1e-6) / 1e9
+    print(f"| frames 1x3x243x768x1344 | frames_to_u8 (BTHWC) | {us:.1f} | - | {gbs:.0f} | "
+          f"{100 * gbs / 8000:.1f} | {100 * gbs / peak:.1f} |", flush=True)
 
 
 def main(argv=None):
