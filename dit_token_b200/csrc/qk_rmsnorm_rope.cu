@@ -40,13 +40,83 @@ __device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
 // or (j, j + D/2) when half-split -- a lane then holds one side of 8 pairs and
 // the lane LPH/2 away holds the other side, fetched with one xor shuffle per
 // element.  MODE none applies the RMSNorm and the weight only.
+//
+// Interleaved (the common case) folds the weight into the rotation: per lane
+// and per pair the four coefficients w0 cos, -w1 sin, w0 sin, w1 cos are formed
+// once per row (for q and for k), so a pair costs 2 multiplies and 2 FMAs plus
+// the RMS scale: (o0, o1) = r * (x0 w0 c - x1 w1 s, x0 w0 s + x1 w1 c).
+
+struct PairCoef {
+    float c00[4], c01[4], c10[4], c11[4];  // o0 = x0 c00 + x1 c01; o1 = x0 c10 + x1 c11
+};
+
+template <int D, int MODE, int NP>
+__device__ __forceinline__ void rms_rotate_heads(uint16_t* base, int H, int sub, float eps, const float (&w)[8],
+                                                 const PairCoef& pc, const float (&cs)[NP], const float (&sn)[NP],
+                                                 bool upper)
+{
+    constexpr int LPH = D / 8;
+    constexpr int HPW = kWarp / LPH;
+    const float inv_d = 1.0f / (float)D;
+    for (int h0 = 0; h0 < H; h0 += HPW * kUnroll) {
+        uint4 xv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int h = h0 + u * HPW + sub;
+            xv[u] = h < H ? ld_stream(base + (int64_t)h * D) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int h = h0 + u * HPW + sub;
+            const uint32_t wd[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+            f32x2 ss2 = f2_make(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const f32x2 xx = f2_from_bf16x2(wd[e]);
+                ss2 = f2_fma(xx, xx, ss2);
+            }
+            const float ss = group_sum<LPH>(ss2.x + ss2.y);  // every lane of the warp takes part
+            const float r = rsqrtf(ss * inv_d + eps);
+            float o[8];
+            if (MODE == kRopeInterleaved) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = bf16_lo(wd[e]), x1 = bf16_hi(wd[e]);
+                    o[2 * e] = r * fmaf(x1, pc.c01[e], x0 * pc.c00[e]);
+                    o[2 * e + 1] = r * fmaf(x1, pc.c11[e], x0 * pc.c10[e]);
+                }
+            } else {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    y[2 * e] = bf16_lo(wd[e]) * (r * w[2 * e]);
+                    y[2 * e + 1] = bf16_hi(wd[e]) * (r * w[2 * e + 1]);
+                }
+                if (MODE == kRopeHalf) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float partner = __shfl_xor_sync(0xffffffffu, y[e], LPH / 2);  // all lanes take part
+                        o[e] = upper ? partner * sn[e % NP] + y[e] * cs[e % NP]
+                                     : y[e] * cs[e % NP] - partner * sn[e % NP];
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = y[e];
+                }
+            }
+            if (h < H)
+                st_stream(base + (int64_t)h * D, pack8(o));
+        }
+    }
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(kCtaThreads)
 qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
 {
     constexpr int LPH = D / 8;          // lanes per head
-    constexpr int HPW = kWarp / LPH;    // heads per warp per step
-    constexpr int NP = MODE == kRopeHalf ? 8 : (MODE == kRopeInterleaved ? 4 : 0);  // pairs per lane
+    constexpr int NP = MODE == kRopeHalf ? 8 : (MODE == kRopeInterleaved ? 4 : 1);  // pairs per lane
     const int lane = threadIdx.x & (kWarp - 1);
     const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     RowSlot s;
@@ -57,8 +127,13 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
     const int li = lane % LPH;   // position inside the head: elements 8*li .. 8*li+7
     const bool upper = MODE == kRopeHalf && li >= LPH / 2;  // holds the j + D/2 side
 
-    float cs[NP > 0 ? NP : 1], sn[NP > 0 ? NP : 1];
-    if (NP > 0) {
+    float cs[NP], sn[NP];
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        cs[e] = 1.f;
+        sn[e] = 0.f;
+    }
+    if (MODE != kRopeNone) {
         // Positions of this row: a row inside the sequence's T x H x W video
         // grid (t-major, then h, then w) is 3D; every later row is 1D, counted
         // from the end of the grid.  Without a grid every row is 1D.
@@ -91,60 +166,25 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
     float wq[8], wk[8];
     unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
     unpack8(ld_shared_vec(p.k_weight + 8 * li), wk);
-
-    const int Hq = p.num_q_heads;
-    const int Htot = Hq + p.num_k_heads;
-    uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride + 8 * li;
-    uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride + 8 * li;
-    const float inv_d = 1.0f / (float)D;
-
-    for (int h0 = 0; h0 < Htot; h0 += HPW * kUnroll) {
-        uint4 xv[kUnroll];
+    PairCoef pq{}, pk{};
+    if (MODE == kRopeInterleaved) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int h = h0 + u * HPW + sub;
-            if (h < Htot)
-                xv[u] = ld_stream(h < Hq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D);
-            else
-                xv[u] = make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int h = h0 + u * HPW + sub;
-            float x[8];
-            unpack8(xv[u], x);
-            float ss = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                ss = fmaf(x[e], x[e], ss);
-            ss = group_sum<LPH>(ss);  // every lane of the warp takes part
-            const float r = rsqrtf(ss * inv_d + p.eps);
-            const bool isq = h < Hq;
-            float y[8], o[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                y[e] = x[e] * r * (isq ? wq[e] : wk[e]);
-            if (MODE == kRopeInterleaved) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    o[2 * e] = y[2 * e] * cs[e] - y[2 * e + 1] * sn[e];
-                    o[2 * e + 1] = y[2 * e] * sn[e] + y[2 * e + 1] * cs[e];
-                }
-            } else if (MODE == kRopeHalf) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float partner = __shfl_xor_sync(0xffffffffu, y[e], LPH / 2);  // all lanes take part
-                    o[e] = upper ? partner * sn[e] + y[e] * cs[e] : y[e] * cs[e] - partner * sn[e];
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    o[e] = y[e];
-            }
-            if (h < Htot)
-                st_stream(isq ? qrow + (int64_t)h * D : krow + (int64_t)(h - Hq) * D, pack8(o));
+        for (int e = 0; e < 4; ++e) {
+            const float c = cs[e % NP], sv = sn[e % NP];
+            pq.c00[e] = wq[2 * e] * c;
+            pq.c01[e] = -wq[2 * e + 1] * sv;
+            pq.c10[e] = wq[2 * e] * sv;
+            pq.c11[e] = wq[2 * e + 1] * c;
+            pk.c00[e] = wk[2 * e] * c;
+            pk.c01[e] = -wk[2 * e + 1] * sv;
+            pk.c10[e] = wk[2 * e] * sv;
+            pk.c11[e] = wk[2 * e + 1] * c;
         }
     }
+    uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride + 8 * li;
+    uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride + 8 * li;
+    rms_rotate_heads<D, MODE, NP>(qrow, p.num_q_heads, sub, p.eps, wq, pq, cs, sn, upper);
+    rms_rotate_heads<D, MODE, NP>(krow, p.num_k_heads, sub, p.eps, wk, pk, cs, sn, upper);
 }
 
 template <int D>
