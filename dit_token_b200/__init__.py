@@ -29,7 +29,7 @@ import torch
 
 __all__ = ["dit_qk_rmsnorm_rope", "dit_adaln_modulate", "dit_gated_residual", "dit_swiglu",
            "dit_gated_residual_adaln", "dit_frames_to_u8",
-           "dit_validate_seqlens", "DitError", "library", "LIB_PATH", "STATUS"]
+           "dit_validate_seqlens", "check_seqlens", "DitError", "library", "LIB_PATH", "STATUS"]
 
 # DIT_TOKEN_LIB may point at another build of the same library.
 LIB_PATH = os.environ.get("DIT_TOKEN_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
@@ -291,3 +291,16 @@ def dit_validate_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tens
         flag = torch.empty(2, dtype=torch.int32, device=cu_seqlens.device)
     _call("dit_validate_seqlens", cs, cp, B, int(num_rows_padded), flag.data_ptr(), _stream(stream))
     return flag
+
+
+def check_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, num_rows_padded: int,
+                  stream=None) -> None:
+    """Validate a packing descriptor on the device and raise DitError
+    (DIT_ERR_SEQLENS) if it is malformed.  Synchronizes with the stream to
+    read the flag, so call it where a host round trip is acceptable (e.g. once
+    per batch layout), not inside a captured or latency-critical sequence."""
+    flag = dit_validate_seqlens(cu_seqlens, cu_seqlens_padded, num_rows_padded, stream=stream)
+    bad, first = (int(v) for v in flag.tolist())
+    if bad:
+        raise DitError("dit_validate_seqlens", 5,
+                       f"{library().dit_status_string(5).decode()}: first bad sequence {first}")

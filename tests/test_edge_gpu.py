@@ -218,3 +218,14 @@ def test_malformed_device_descriptors_are_skipped_and_flagged():
     bad2 = dit.dit_validate_seqlens(cs2, cp2, 16)
     torch.cuda.synchronize()
     assert good.tolist()[0] == 0 and bad2.tolist() == [1, 1]
+
+
+def test_check_seqlens_raises_on_malformed_descriptors():
+    ok_cs = torch.tensor([0, 6, 12], dtype=torch.int32, device="cuda")
+    ok_cp = torch.tensor([0, 8, 16], dtype=torch.int32, device="cuda")
+    dit.check_seqlens(ok_cs, ok_cp, 16)
+    with pytest.raises(dit.DitError) as e:
+        dit.check_seqlens(torch.tensor([0, 9, 12], dtype=torch.int32, device="cuda"), ok_cp, 16)
+    assert e.value.status == 5
+    with pytest.raises(dit.DitError):
+        dit.check_seqlens(ok_cs, ok_cp, 12)   # the descriptor runs past the buffer
