@@ -49,6 +49,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_gated_residual_adaln.argtypes = [
             u16p, i64, u16p, i64, u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64,
             u16p, i64, u16p, i64, f64p, i64p, i64]
+        vp = ctypes.c_void_p
+        L.oracle_adaln_modulate_ex.argtypes = [
+            u16p, i64, vp, vp, i64, i32, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
+        L.oracle_gated_residual_ex.argtypes = [
+            u16p, i64, u16p, i64, vp, i64, i32, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
+        L.oracle_gated_residual_adaln_ex.argtypes = [
+            u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i32p, i32, i64, i32, f64,
+            u16p, i64, u16p, i64, f64p, i64p, i64]
         L.oracle_swiglu.argtypes = [
             u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
         L.oracle_frames_to_u8.argtypes = [ctypes.POINTER(ctypes.c_float), i64, i64, i64, i64, i64, i32,
@@ -56,6 +64,7 @@ def lib() -> ctypes.CDLL:
         for name in ("oracle_qk_rmsnorm_rope", "oracle_qk_rmsnorm_rope_ex", "oracle_adaln_modulate",
                      "oracle_frames_to_u8",
                      "oracle_gated_residual", "oracle_gated_residual_adaln", "oracle_swiglu",
+                     "oracle_adaln_modulate_ex", "oracle_gated_residual_ex", "oracle_gated_residual_adaln_ex",
                      "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -99,6 +108,21 @@ def _flat_view(a, row_stride, rows_padded):
     if row_stride is None:
         row_stride = int(np.prod(a.shape[1:])) if a.ndim > 1 else 1
     return a, row_stride
+
+
+def _mod(a):
+    """Per-sequence modulation vectors: raw bf16 bits (uint16) or fp32 values.
+    Returns (contiguous array, is_fp32)."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray(a), 0
+    if a.dtype == np.float32:
+        return np.ascontiguousarray(a), 1
+    raise TypeError(f"modulation vectors must be uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+def _vptr(a):
+    return ctypes.c_void_p(a.ctypes.data)
 
 
 def bf16_to_f64(bits: int) -> float:
@@ -185,12 +209,14 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
     if out is None:
         out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
     o64 = np.full(out.shape, np.nan) if want_f64 else None
-    sh = np.ascontiguousarray(_u16(shift))
-    sc = np.ascontiguousarray(_u16(scale))
+    sh, f1 = _mod(shift)
+    sc, f2 = _mod(scale)
+    if f1 != f2:
+        raise TypeError("shift and scale must have the same dtype")
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_adaln_modulate(
-        _ptr(x, ctypes.c_uint16), xs, _ptr(sh, ctypes.c_uint16), _ptr(sc, ctypes.c_uint16), mss,
+    rc = lib().oracle_adaln_modulate_ex(
+        _ptr(x, ctypes.c_uint16), xs, _vptr(sh), _vptr(sc), mss, f1,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "adaln_modulate")
@@ -209,11 +235,11 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
     if out is None:
         out = np.array(x if out_init is None else out_init, dtype=np.uint16, copy=True)
     o64 = np.full(out.shape, np.nan) if want_f64 else None
-    g = np.ascontiguousarray(_u16(gate))
+    g, gf = _mod(gate)
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_gated_residual(
-        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _ptr(g, ctypes.c_uint16), gss,
+    rc = lib().oracle_gated_residual_ex(
+        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss, gf,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "gated_residual")
@@ -236,15 +262,17 @@ def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded
     if norm_out is None:
         norm_out = np.array(x if norm_init is None else norm_init, dtype=np.uint16, copy=True)
     n64 = np.full(norm_out.shape, np.nan) if want_f64 else None
-    g = np.ascontiguousarray(_u16(gate))
-    sh = np.ascontiguousarray(_u16(shift))
-    sc = np.ascontiguousarray(_u16(scale))
+    g, f0 = _mod(gate)
+    sh, f1 = _mod(shift)
+    sc, f2 = _mod(scale)
+    if not (f0 == f1 == f2):
+        raise TypeError("gate, shift and scale must have the same dtype")
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_gated_residual_adaln(
-        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _ptr(g, ctypes.c_uint16), gss,
-        _ptr(sh, ctypes.c_uint16), _ptr(sc, ctypes.c_uint16), mss,
+    rc = lib().oracle_gated_residual_adaln_ex(
+        _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss,
+        _vptr(sh), _vptr(sc), mss, f1,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(res_out, ctypes.c_uint16), xs, _ptr(norm_out, ctypes.c_uint16), xs, _ptr(n64, ctypes.c_double),
         _ptr(r, ctypes.c_int64), nr)

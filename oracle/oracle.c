@@ -68,6 +68,15 @@ uint16_t oracle_f64_to_bf16(double x)
 
 static double ld(const uint16_t* p) { return oracle_bf16_to_f64(*p); }
 
+/* Element idx of a per-sequence modulation vector stored as bf16 bits or as
+ * fp32 (f32 != 0), widened exactly. */
+static double ldm(const void* base, int64_t idx, int f32)
+{
+    if (f32)
+        return (double)((const float*)base)[idx];
+    return oracle_bf16_to_f64(((const uint16_t*)base)[idx]);
+}
+
 /* -------------------------------------------------------- packed rows */
 
 /* The padded buffer holds num_seqs sequences; sequence b owns padded rows
@@ -282,6 +291,19 @@ int oracle_adaln_modulate(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_adaln_modulate_ex(x, x_row_stride, shift, scale, mod_seq_stride, 0, cu_seqlens,
+                                    cu_seqlens_padded, num_seqs, num_rows_padded, hidden, eps, out,
+                                    out_row_stride, out_f64, rows, num_rows);
+}
+
+int oracle_adaln_modulate_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!x || !shift || !scale || !out || hidden <= 0)
         return -1;
     if (x_row_stride < hidden || out_row_stride < hidden || mod_seq_stride < 0)
@@ -299,8 +321,7 @@ int oracle_adaln_modulate(
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
         const uint16_t* xr = x + row * x_row_stride;
-        const uint16_t* sh = shift + (int64_t)b * mod_seq_stride;
-        const uint16_t* sc = scale + (int64_t)b * mod_seq_stride;
+        const int64_t mb = (int64_t)b * mod_seq_stride;
         /* LayerNorm without affine: mean, then the biased variance about it. */
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
@@ -314,7 +335,7 @@ int oracle_adaln_modulate(
         /* Modulation: x_hat * (1 + scale) + shift. */
         for (int32_t c = 0; c < hidden; ++c) {
             double xhat = (ld(&xr[c]) - mean) * inv_std;
-            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);
+            double v = xhat * (1.0 + ldm(scale, mb + c, mod_f32)) + ldm(shift, mb + c, mod_f32);
             put(out, out_f64, row * out_row_stride + c, v);
         }
     }
@@ -327,6 +348,20 @@ int oracle_gated_residual(
     const uint16_t* x, int64_t x_row_stride,
     const uint16_t* y, int64_t y_row_stride,
     const uint16_t* gate, int64_t gate_seq_stride,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
+    return oracle_gated_residual_ex(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, 0, cu_seqlens,
+                                    cu_seqlens_padded, num_seqs, num_rows_padded, hidden, out, out_row_stride,
+                                    out_f64, rows, num_rows);
+}
+
+int oracle_gated_residual_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
@@ -348,9 +383,9 @@ int oracle_gated_residual(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const uint16_t* g = gate + (int64_t)b * gate_seq_stride;
+        const int64_t gb = (int64_t)b * gate_seq_stride;
         for (int32_t c = 0; c < hidden; ++c) {
-            double v = ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]);
+            double v = ld(&x[row * x_row_stride + c]) + ldm(gate, gb + c, gate_f32) * ld(&y[row * y_row_stride + c]);
             put(out, out_f64, row * out_row_stride + c, v);
         }
     }
@@ -376,6 +411,23 @@ int oracle_gated_residual_adaln(
     uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_gated_residual_adaln_ex(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, shift, scale,
+                                          mod_seq_stride, 0, cu_seqlens, cu_seqlens_padded, num_seqs,
+                                          num_rows_padded, hidden, eps, res_out, res_row_stride, norm_out,
+                                          norm_row_stride, norm_out_f64, rows, num_rows);
+}
+
+int oracle_gated_residual_adaln_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!x || !y || !gate || !shift || !scale || !res_out || !norm_out || hidden <= 0)
         return -1;
     if (x_row_stride < hidden || y_row_stride < hidden || res_row_stride < hidden || norm_row_stride < hidden ||
@@ -393,16 +445,15 @@ int oracle_gated_residual_adaln(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const uint16_t* g = gate + (int64_t)b * gate_seq_stride;
+        const int64_t gb = (int64_t)b * gate_seq_stride;
         uint16_t* rr = res_out + row * res_row_stride;
         /* step 1: residual update, stored as bf16 */
         for (int32_t c = 0; c < hidden; ++c) {
-            double v = ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]);
+            double v = ld(&x[row * x_row_stride + c]) + ldm(gate, gb + c, mod_f32) * ld(&y[row * y_row_stride + c]);
             rr[c] = oracle_f64_to_bf16(v);
         }
         /* step 2: adaLN of the stored residual */
-        const uint16_t* sh = shift + (int64_t)b * mod_seq_stride;
-        const uint16_t* sc = scale + (int64_t)b * mod_seq_stride;
+        const int64_t mb = (int64_t)b * mod_seq_stride;
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
             mean += ld(&rr[c]);
@@ -414,7 +465,7 @@ int oracle_gated_residual_adaln(
         double inv_std = 1.0 / sqrt(var + eps);
         for (int32_t c = 0; c < hidden; ++c) {
             double xhat = (ld(&rr[c]) - mean) * inv_std;
-            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);
+            double v = xhat * (1.0 + ldm(scale, mb + c, mod_f32)) + ldm(shift, mb + c, mod_f32);
             put(norm_out, norm_out_f64, row * norm_row_stride + c, v);
         }
     }

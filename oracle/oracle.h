@@ -125,6 +125,34 @@ int oracle_gated_residual_adaln(
     uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
     const int64_t* rows, int64_t num_rows);
 
+/* The modulated ops with their per-sequence vectors (gate, shift, scale) in
+ * either bf16 bits (f32 == 0) or fp32 (f32 != 0); everything else as above. */
+int oracle_adaln_modulate_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows);
+int oracle_gated_residual_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows);
+int oracle_gated_residual_adaln_ex(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows);
+
 /* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)). */
 int oracle_swiglu(
     const uint16_t* a, int64_t a_row_stride,

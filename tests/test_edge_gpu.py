@@ -229,3 +229,23 @@ def test_check_seqlens_raises_on_malformed_descriptors():
     assert e.value.status == 5
     with pytest.raises(dit.DitError):
         dit.check_seqlens(ok_cs, ok_cp, 12)   # the descriptor runs past the buffer
+
+
+def test_gqa_at_scale_and_thousands_of_sequences():
+    # 40 query heads sharing 8 key heads over a 16k-row batch of the big shapes
+    lengths = [4000, 7000, 5000]
+    padded = [-(-L // 128) * 128 for L in lengths]
+    w = W.custom("gqa", lengths, padded, hidden=5120, num_q_heads=40, num_k_heads=8, head_dim=128, inner=8,
+                 grids=[(L // 1008, 24, 42) for L in lengths], sections=(44, 42, 42), seed=21)
+    rows = W.sample_rows(w, per_seq=48)
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp)
+    qo, ko = P.oracle_qk(w, inp, rows)
+    P.assert_close(P.gather_rows(q, rows), qo[rows], "q gqa")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], "k gqa")
+    # 2500 sequences: the sequence search takes three 32-way levels
+    rng = np.random.default_rng(5)
+    lengths = rng.integers(0, 6, 2500)
+    padded = [int(L) + int(rng.integers(0, 3)) for L in lengths]
+    w = W.custom("many2", lengths, padded, hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64, seed=3)
+    all_ops_full(w)

@@ -17,7 +17,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
         "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py",
-        "tests/test_oracle_frames.py", "tests/test_oracle_rope_modes.py"]
+        "tests/test_oracle_frames.py", "tests/test_oracle_rope_modes.py",
+        "tests/test_oracle_modulation_f32.py"]
 
 # (name, original text, planted mistake)
 MUTANTS = [
@@ -35,12 +36,15 @@ MUTANTS = [
     ("rope_3d_h_index", "pos3[1] = (r / W) % H;", "pos3[1] = (r / H) % W;"),
     ("rope_tail_position", "pos1 = r - thw;", "pos1 = r;"),
     ("rope_k_uses_q_weight", "rmsnorm_rope_head(k + off, k_weight,", "rmsnorm_rope_head(k + off, q_weight,"),
-    ("adaln_scale_without_one", "xhat * (1.0 + ld(&sc[c]))", "xhat * ld(&sc[c])"),
+    ("adaln_scale_without_one", "xhat * (1.0 + ldm(scale, mb + c, mod_f32))", "xhat * ldm(scale, mb + c, mod_f32)"),
     ("adaln_unbiased_variance", "var /= (double)hidden;", "var /= (double)(hidden - 1);"),
-    ("adaln_shift_scale_swapped", "double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);",
-     "double v = xhat * (1.0 + ld(&sh[c])) + ld(&sc[c]);"),
-    ("gate_dropped", "ld(&g[c]) * ld(&y[row * y_row_stride + c])", "ld(&y[row * y_row_stride + c])"),
-    ("gate_not_per_sequence", "gate + (int64_t)b * gate_seq_stride", "gate"),
+    ("adaln_shift_scale_swapped", "xhat * (1.0 + ldm(scale, mb + c, mod_f32)) + ldm(shift, mb + c, mod_f32)",
+     "xhat * (1.0 + ldm(shift, mb + c, mod_f32)) + ldm(scale, mb + c, mod_f32)"),
+    ("gate_dropped", "ldm(gate, gb + c, gate_f32) * ld(&y[row * y_row_stride + c])",
+     "ld(&y[row * y_row_stride + c])"),
+    ("fused_gate_dropped", "ldm(gate, gb + c, mod_f32) * ld(&y[row * y_row_stride + c])",
+     "ld(&y[row * y_row_stride + c])"),
+    ("gate_not_per_sequence", "const int64_t gb = (int64_t)b * gate_seq_stride;", "const int64_t gb = 0;"),
     ("silu_sign", "exp(-av)", "exp(av)"),
     ("swiglu_operands_transposed", "double silu = av / (1.0 + exp(-av));\n            put(out, out_f64, row * out_row_stride + c, silu * bv);",
      "double silu = bv / (1.0 + exp(-bv));\n            put(out, out_f64, row * out_row_stride + c, silu * av);"),
@@ -48,8 +52,10 @@ MUTANTS = [
     ("padding_row_read", "if (r < len) {", "if (r <= len) {"),
     ("fused_mean_over_x_not_residual", "mean += ld(&rr[c]);", "mean += ld(&x[row * x_row_stride + c]);"),
     ("fused_residual_not_rounded_before_norm",
-     "double xhat = (ld(&rr[c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out",
-     "double xhat = (ld(&x[row * x_row_stride + c]) + ld(&g[c]) * ld(&y[row * y_row_stride + c]) - mean) * inv_std;\n            double v = xhat * (1.0 + ld(&sc[c])) + ld(&sh[c]);\n            put(norm_out"),
+     "double xhat = (ld(&rr[c]) - mean) * inv_std;",
+     "double xhat = (ld(&x[row * x_row_stride + c]) + ldm(gate, gb + c, mod_f32) * ld(&y[row * y_row_stride + c]) - mean) * inv_std;"),
+    ("fp32_modulation_read_as_bf16", "return (double)((const float*)base)[idx];",
+     "return oracle_bf16_to_f64(((const uint16_t*)base)[idx]);"),
     ("frames_truncates", "return (uint8_t)nearbyintf(u);", "return (uint8_t)u;"),
     ("frames_no_clamp_top", "if (u >= 255.0f)\n        return 255;", ""),
     ("frames_wrong_layout", "? (((b * frames + t) * height + h) * width + w) * channels + c",
