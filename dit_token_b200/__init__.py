@@ -58,10 +58,16 @@ _SIGNATURES = {
     "dit_qk_rmsnorm_rope_ex": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
                                _VP, _I32, _I32, _I32, _F32, _F32, _I32, _VP],
     "dit_adaln_modulate": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _VP],
+    "dit_adaln_modulate_ex": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _I32,
+                              _VP],
     "dit_gated_residual": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
+    "dit_gated_residual_ex": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _I32,
+                              _VP],
     "dit_swiglu": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _VP],
     "dit_gated_residual_adaln": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _I64, _VP, _I64,
                                  _VP, _VP, _I32, _I64, _I32, _F32, _VP],
+    "dit_gated_residual_adaln_ex": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _I64, _VP, _I64,
+                                    _VP, _VP, _I32, _I64, _I32, _F32, _I32, _VP],
     "dit_validate_seqlens": [_VP, _VP, _I32, _I64, _VP, _VP],
     "dit_frames_to_u8": [_VP, _I64, _I64, _I64, _I64, _I64, _I32, _VP, _VP],
     "dit_status_string": [_I32],
@@ -127,14 +133,24 @@ def _vec(t: torch.Tensor, what: str) -> int:
     return t.data_ptr()
 
 
+# element-type codes of the per-sequence vectors (DIT_DTYPE_* in dit_token.h)
+_DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
+
+
 def _seq_vectors(t: torch.Tensor, hidden: int, what: str) -> tuple:
-    """(pointer, per-sequence stride) of per-sequence vectors [num_seqs, hidden]
-    (any sequence stride, contiguous last axis)."""
-    if t.dtype != torch.bfloat16 or not t.is_cuda:
-        raise TypeError(f"{what}: expected a bfloat16 CUDA tensor")
+    """(pointer, per-sequence stride, dtype code) of per-sequence vectors
+    [num_seqs, hidden], bf16 or fp32 (any sequence stride, contiguous last axis)."""
+    if t.dtype not in _DTYPE_CODES or not t.is_cuda:
+        raise TypeError(f"{what}: expected a bfloat16 or float32 CUDA tensor")
     if t.dim() != 2 or t.size(1) != hidden or (t.stride(1) != 1 and hidden > 1):
         raise ValueError(f"{what}: expected [num_seqs, {hidden}] with a contiguous last axis")
-    return t.data_ptr(), t.stride(0)
+    return t.data_ptr(), t.stride(0), _DTYPE_CODES[t.dtype]
+
+
+def _one_dtype(codes, what: str) -> int:
+    if len(set(codes)) != 1:
+        raise TypeError(f"{what} must all be bfloat16 or all float32")
+    return codes[0]
 
 
 def _packing(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor):
@@ -188,37 +204,46 @@ def dit_adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor
 
     x: [rows, hidden]; shift, scale: [num_seqs, hidden] (any sequence stride,
     e.g. slices of a [num_seqs, 6, hidden] modulation tensor -- both must
-    share it).  ``out`` may be x; if None a new tensor is returned whose
-    padding rows are left uninitialised."""
+    share it), both bf16 (dit_adaln_modulate) or both fp32
+    (dit_adaln_modulate_ex).  ``out`` may be x; if None a new tensor is
+    returned whose padding rows are left uninitialised."""
     hidden = x.size(-1)
     if out is None:
         out = torch.empty_like(x)
     xp, xs = _rows(x, "x")
     op, os_ = _rows(out, "out")
-    shp, sst = _seq_vectors(shift, hidden, "shift")
-    scp, cst = _seq_vectors(scale, hidden, "scale")
+    shp, sst, shd = _seq_vectors(shift, hidden, "shift")
+    scp, cst, scd = _seq_vectors(scale, hidden, "scale")
+    dt = _one_dtype((shd, scd), "shift and scale")
     cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
     if B > 1 and sst != cst:
         raise ValueError("shift and scale must share one sequence stride")
-    _call("dit_adaln_modulate", xp, xs, op, os_, shp, scp, sst if B > 1 else hidden, cs, cp, B, x.size(0),
-          hidden, float(eps), _stream(stream))
+    args = (xp, xs, op, os_, shp, scp, sst if B > 1 else hidden, cs, cp, B, x.size(0), hidden, float(eps))
+    if dt == 0:
+        _call("dit_adaln_modulate", *args, _stream(stream))
+    else:
+        _call("dit_adaln_modulate_ex", *args, dt, _stream(stream))
     return out
 
 
 def dit_gated_residual(x: torch.Tensor, y: torch.Tensor, gate: torch.Tensor,
                        cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, *,
                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """out = x + gate_b * y on valid rows (``out`` may be x)."""
+    """out = x + gate_b * y on valid rows (``out`` may be x).  gate: bf16
+    (dit_gated_residual) or fp32 (dit_gated_residual_ex) [num_seqs, hidden]."""
     hidden = x.size(-1)
     if out is None:
         out = torch.empty_like(x)
     xp, xs = _rows(x, "x")
     yp, ys = _rows(y, "y")
     op, os_ = _rows(out, "out")
-    gp, gst = _seq_vectors(gate, hidden, "gate")
+    gp, gst, dt = _seq_vectors(gate, hidden, "gate")
     cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
-    _call("dit_gated_residual", xp, xs, yp, ys, gp, gst if B > 1 else hidden, op, os_, cs, cp, B,
-          x.size(0), hidden, _stream(stream))
+    args = (xp, xs, yp, ys, gp, gst if B > 1 else hidden, op, os_, cs, cp, B, x.size(0), hidden)
+    if dt == 0:
+        _call("dit_gated_residual", *args, _stream(stream))
+    else:
+        _call("dit_gated_residual_ex", *args, dt, _stream(stream))
     return out
 
 
@@ -227,7 +252,9 @@ def dit_gated_residual_adaln(x: torch.Tensor, y: torch.Tensor, gate: torch.Tenso
                              res_out: Optional[torch.Tensor] = None, norm_out: Optional[torch.Tensor] = None,
                              eps: float = 1e-6, stream=None):
     """res = x + gate_b * y; norm = LayerNorm(res) * (1 + scale_b) + shift_b,
-    on valid rows, in one pass.  ``res_out`` may be x.  Returns (res, norm)."""
+    on valid rows, in one pass.  ``res_out`` may be x.  gate, shift and scale
+    all bf16 (dit_gated_residual_adaln) or all fp32 (dit_gated_residual_adaln_ex).
+    Returns (res, norm)."""
     hidden = x.size(-1)
     if res_out is None:
         res_out = torch.empty_like(x)
@@ -237,14 +264,19 @@ def dit_gated_residual_adaln(x: torch.Tensor, y: torch.Tensor, gate: torch.Tenso
     yp, ys = _rows(y, "y")
     rp, rs = _rows(res_out, "res_out")
     np_, ns = _rows(norm_out, "norm_out")
-    gp, gst = _seq_vectors(gate, hidden, "gate")
-    shp, sst = _seq_vectors(shift, hidden, "shift")
-    scp, cst = _seq_vectors(scale, hidden, "scale")
+    gp, gst, gd = _seq_vectors(gate, hidden, "gate")
+    shp, sst, shd = _seq_vectors(shift, hidden, "shift")
+    scp, cst, scd = _seq_vectors(scale, hidden, "scale")
+    dt = _one_dtype((gd, shd, scd), "gate, shift and scale")
     cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
     if B > 1 and sst != cst:
         raise ValueError("shift and scale must share one sequence stride")
-    _call("dit_gated_residual_adaln", xp, xs, yp, ys, gp, gst if B > 1 else hidden, shp, scp,
-          sst if B > 1 else hidden, rp, rs, np_, ns, cs, cp, B, x.size(0), hidden, float(eps), _stream(stream))
+    args = (xp, xs, yp, ys, gp, gst if B > 1 else hidden, shp, scp, sst if B > 1 else hidden, rp, rs, np_, ns,
+            cs, cp, B, x.size(0), hidden, float(eps))
+    if dt == 0:
+        _call("dit_gated_residual_adaln", *args, _stream(stream))
+    else:
+        _call("dit_gated_residual_adaln_ex", *args, dt, _stream(stream))
     return res_out, norm_out
 
 

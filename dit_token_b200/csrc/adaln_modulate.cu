@@ -76,25 +76,23 @@ __device__ __forceinline__ uint4 modulate8(uint4 x, f32x2 r2, f32x2 b2, const f3
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// A = 1 + scale and B = shift of vector j, from global bf16.
-__device__ __forceinline__ void mod_from_global(const uint16_t* sh, const uint16_t* sc, int j, f32x2 (&A)[4],
+// A = 1 + scale and B = shift of the 8 elements at element `elem` of a
+// sequence's vectors, from global memory (bf16 or fp32).
+template <bool F32>
+__device__ __forceinline__ void mod_from_global(const void* shift, const void* scale, int64_t elem, f32x2 (&A)[4],
                                                 f32x2 (&B)[4])
 {
-    const uint4 shv = ld_shared_vec(sh + 8 * j);
-    const uint4 scv = ld_shared_vec(sc + 8 * j);
-    const uint32_t hw[4] = {shv.x, shv.y, shv.z, shv.w};
-    const uint32_t cw[4] = {scv.x, scv.y, scv.z, scv.w};
+    vec8_pairs<F32>(scale, elem, A);
+    vec8_pairs<F32>(shift, elem, B);
     const f32x2 one2 = f2_make(1.f, 1.f);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        A[e] = f2_add(f2_from_bf16x2(cw[e]), one2);
-        B[e] = f2_from_bf16x2(hw[e]);
-    }
+    for (int e = 0; e < 4; ++e)
+        A[e] = f2_add(A[e], one2);
 }
 
 // ------------------------------------------------------------ warp per row
 
-template <int VPT>
+template <int VPT, bool F32>
 __global__ void __launch_bounds__(kCtaThreads)
 adaln_warp_kernel(const AdalnParams p, int slots)
 {
@@ -126,17 +124,16 @@ adaln_warp_kernel(const AdalnParams p, int slots)
                 continue;  // uniform
             float* A = mod_smem + (size_t)sidx * 2 * C;
             float* B = A + C;
-            const uint16_t* sh = p.shift + (int64_t)b * p.mod_seq_stride;
-            const uint16_t* sc = p.scale + (int64_t)b * p.mod_seq_stride;
+            const int64_t moff = (int64_t)b * p.mod_seq_stride;
             for (int j = tid; j < nvec; j += kCtaThreads) {
-                float a[8], bb[8];
-                unpack8(ld_shared_vec(sc + 8 * j), a);
-                unpack8(ld_shared_vec(sh + 8 * j), bb);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    A[8 * j + e] = 1.0f + a[e];
-                    B[8 * j + e] = bb[e];
-                }
+                f32x2 a[4], bb[4];
+                mod_from_global<F32>(p.shift, p.scale, moff + 8 * j, a, bb);
+                float4* A4 = reinterpret_cast<float4*>(A + 8 * j);
+                float4* B4 = reinterpret_cast<float4*>(B + 8 * j);
+                A4[0] = make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
+                A4[1] = make_float4(a[2].x, a[2].y, a[3].x, a[3].y);
+                B4[0] = make_float4(bb[0].x, bb[0].y, bb[1].x, bb[1].y);
+                B4[1] = make_float4(bb[2].x, bb[2].y, bb[3].x, bb[3].y);
             }
         }
         __syncthreads();
@@ -190,14 +187,13 @@ adaln_warp_kernel(const AdalnParams p, int slots)
                 }
             }
         } else {
-            const uint16_t* sh = p.shift + (int64_t)seq * p.mod_seq_stride;
-            const uint16_t* sc = p.scale + (int64_t)seq * p.mod_seq_stride;
+            const int64_t moff = (int64_t)seq * p.mod_seq_stride;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int j = i * kWarp + lane;
                 if (j < nvec) {
                     f32x2 Av[4], Bv[4];
-                    mod_from_global(sh, sc, j, Av, Bv);
+                    mod_from_global<F32>(p.shift, p.scale, moff + 8 * j, Av, Bv);
                     st_stream(orow + 8 * kWarp * i, modulate8(xv[i], r2, b2, Av, Bv));
                 }
             }
@@ -205,33 +201,39 @@ adaln_warp_kernel(const AdalnParams p, int slots)
     }
 }
 
-template <int VPT>
-cudaError_t launch_warp(const AdalnParams& p, cudaStream_t stream)
+template <int VPT, bool F32>
+cudaError_t launch_warp_t(const AdalnParams& p, cudaStream_t stream)
 {
     const size_t slot_bytes = (size_t)2 * p.hidden * sizeof(float);
     const int slots = 2 * slot_bytes <= (size_t)kSmemBudget ? 2 : (slot_bytes <= (size_t)kSmemBudget ? 1 : 0);
     const size_t smem = slots * slot_bytes;
     cudaError_t e;
     if (smem > 48 * 1024 &&
-        (e = cudaFuncSetAttribute(adaln_warp_kernel<VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
+        (e = cudaFuncSetAttribute(adaln_warp_kernel<VPT, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
         return e;
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_warp_kernel<VPT>, kCtaThreads, smem)) !=
-            cudaSuccess)
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_warp_kernel<VPT, F32>, kCtaThreads,
+                                                           smem)) != cudaSuccess)
         return e;
     const long long want = (long long)sms * (per_sm > 0 ? per_sm : 1);
     const long long rows_cap = (p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta;
     const unsigned grid = (unsigned)(want < rows_cap ? want : rows_cap);
-    adaln_warp_kernel<VPT><<<grid, kCtaThreads, smem, stream>>>(p, slots);
+    adaln_warp_kernel<VPT, F32><<<grid, kCtaThreads, smem, stream>>>(p, slots);
     return cudaGetLastError();
+}
+
+template <int VPT>
+cudaError_t launch_warp(const AdalnParams& p, cudaStream_t stream)
+{
+    return p.mod_f32 ? launch_warp_t<VPT, true>(p, stream) : launch_warp_t<VPT, false>(p, stream);
 }
 
 // ------------------------------------------------------------ team per row
 
-template <int VPT, int TEAM>
+template <int VPT, int TEAM, bool F32>
 __global__ void __launch_bounds__(kCtaThreads, MinCtas<VPT>::value)
 adaln_team_kernel(const AdalnParams p)
 {
@@ -266,15 +268,14 @@ adaln_team_kernel(const AdalnParams p)
     const f32x2 r2 = f2_make(rstd, rstd);
     const float nb = -m.mean * rstd;
     const f32x2 b2 = f2_make(nb, nb);
-    const uint16_t* sh = p.shift + (int64_t)s.seq * p.mod_seq_stride;
-    const uint16_t* sc = p.scale + (int64_t)s.seq * p.mod_seq_stride;
+    const int64_t moff = (int64_t)s.seq * p.mod_seq_stride;
     uint16_t* orow = p.out + (int64_t)s.row * p.out_row_stride;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
             f32x2 Av[4], Bv[4];
-            mod_from_global(sh, sc, j, Av, Bv);
+            mod_from_global<F32>(p.shift, p.scale, moff + 8 * j, Av, Bv);
             st_stream(orow + 8 * j, modulate8(xv[i], r2, b2, Av, Bv));
         }
     }
@@ -287,14 +288,22 @@ cudaError_t launch_team(const AdalnParams& p, cudaStream_t stream)
     const int vpt = (nvec + TEAM * kWarp - 1) / (TEAM * kWarp);
     const int rows_per_cta = kWarpsPerCta / TEAM;
     const unsigned grid = (unsigned)((p.pk.num_rows_padded + rows_per_cta - 1) / rows_per_cta);
+#define DIT_TEAM_CASE(V)                                                                                     \
+    case V:                                                                                                  \
+        if (p.mod_f32)                                                                                       \
+            adaln_team_kernel<V, TEAM, true><<<grid, kCtaThreads, 0, stream>>>(p);                           \
+        else                                                                                                 \
+            adaln_team_kernel<V, TEAM, false><<<grid, kCtaThreads, 0, stream>>>(p);                          \
+        break;
     switch (vpt) {
-    case 4: adaln_team_kernel<4, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case 5: adaln_team_kernel<5, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case 6: adaln_team_kernel<6, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case 7: adaln_team_kernel<7, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case 8: adaln_team_kernel<8, TEAM><<<grid, kCtaThreads, 0, stream>>>(p); break;
+        DIT_TEAM_CASE(4)
+        DIT_TEAM_CASE(5)
+        DIT_TEAM_CASE(6)
+        DIT_TEAM_CASE(7)
+        DIT_TEAM_CASE(8)
     default: return cudaErrorInvalidValue;
     }
+#undef DIT_TEAM_CASE
     return cudaGetLastError();
 }
 

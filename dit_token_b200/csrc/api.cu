@@ -21,6 +21,12 @@ thread_local int32_t g_last_cuda_error = 0;
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool mult8(int64_t v) { return (v & 7) == 0; }
 
+// A per-sequence vector stride keeps every sequence's vector 16-byte aligned:
+// a multiple of 8 bf16 or of 4 fp32 elements.
+bool mod_stride_ok(int64_t v, bool f32) { return f32 ? (v & 3) == 0 : mult8(v); }
+
+bool known_dtype(int32_t d) { return d == DIT_DTYPE_BF16 || d == DIT_DTYPE_F32; }
+
 dit_status from_cuda(cudaError_t e)
 {
     if (e == cudaSuccess)
@@ -147,6 +153,20 @@ dit_status dit_adaln_modulate(const void* x, int64_t x_row_stride, void* out, in
                               int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
                               void* stream)
 {
+    return dit_adaln_modulate_ex(x, x_row_stride, out, out_row_stride, shift, scale, mod_seq_stride, cu_seqlens,
+                                 cu_seqlens_padded, num_seqs, num_rows_padded, hidden, eps, DIT_DTYPE_BF16,
+                                 stream);
+}
+
+dit_status dit_adaln_modulate_ex(const void* x, int64_t x_row_stride, void* out, int64_t out_row_stride,
+                                 const void* shift, const void* scale, int64_t mod_seq_stride,
+                                 const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                 int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
+                                 int32_t mod_dtype, void* stream)
+{
+    if (!known_dtype(mod_dtype))
+        return DIT_ERR_UNSUPPORTED;
+    const bool f32 = mod_dtype == DIT_DTYPE_F32;
     bool empty = false;
     dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
     if (st != DIT_OK)
@@ -161,12 +181,12 @@ dit_status dit_adaln_modulate(const void* x, int64_t x_row_stride, void* out, in
     if (!x || !out || !shift || !scale)
         return DIT_ERR_NULL;
     if (!aligned16(x) || !aligned16(out) || !aligned16(shift) || !aligned16(scale) || !mult8(hidden) ||
-        !mult8(x_row_stride) || !mult8(out_row_stride) || !mult8(mod_seq_stride))
+        !mult8(x_row_stride) || !mult8(out_row_stride) || !mod_stride_ok(mod_seq_stride, f32))
         return DIT_ERR_ALIGN;
-    dit::AdalnParams p{static_cast<const uint16_t*>(x), static_cast<uint16_t*>(out),
-                       static_cast<const uint16_t*>(shift), static_cast<const uint16_t*>(scale),
+    dit::AdalnParams p{static_cast<const uint16_t*>(x), static_cast<uint16_t*>(out), shift, scale,
                        x_row_stride, out_row_stride, mod_seq_stride,
-                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps};
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps,
+                       f32 ? 1 : 0};
     return from_cuda(dit::launch_adaln_modulate(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -175,6 +195,20 @@ dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const void* y
                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
                               int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, void* stream)
 {
+    return dit_gated_residual_ex(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, out, out_row_stride,
+                                 cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, hidden, DIT_DTYPE_BF16,
+                                 stream);
+}
+
+dit_status dit_gated_residual_ex(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                                 const void* gate, int64_t gate_seq_stride, void* out, int64_t out_row_stride,
+                                 const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                 int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, int32_t gate_dtype,
+                                 void* stream)
+{
+    if (!known_dtype(gate_dtype))
+        return DIT_ERR_UNSUPPORTED;
+    const bool f32 = gate_dtype == DIT_DTYPE_F32;
     bool empty = false;
     dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
     if (st != DIT_OK)
@@ -187,12 +221,12 @@ dit_status dit_gated_residual(const void* x, int64_t x_row_stride, const void* y
     if (!x || !y || !gate || !out)
         return DIT_ERR_NULL;
     if (!aligned16(x) || !aligned16(y) || !aligned16(gate) || !aligned16(out) || !mult8(hidden) ||
-        !mult8(x_row_stride) || !mult8(y_row_stride) || !mult8(out_row_stride) || !mult8(gate_seq_stride))
+        !mult8(x_row_stride) || !mult8(y_row_stride) || !mult8(out_row_stride) ||
+        !mod_stride_ok(gate_seq_stride, f32))
         return DIT_ERR_ALIGN;
-    dit::GatedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y),
-                       static_cast<const uint16_t*>(gate), static_cast<uint16_t*>(out),
-                       x_row_stride, y_row_stride, gate_seq_stride, out_row_stride,
-                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden};
+    dit::GatedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y), gate,
+                       static_cast<uint16_t*>(out), x_row_stride, y_row_stride, gate_seq_stride, out_row_stride,
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, f32 ? 1 : 0};
     return from_cuda(dit::launch_gated_residual(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -204,6 +238,24 @@ dit_status dit_gated_residual_adaln(const void* x, int64_t x_row_stride, const v
                                     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
                                     void* stream)
 {
+    return dit_gated_residual_adaln_ex(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, shift, scale,
+                                       mod_seq_stride, res_out, res_row_stride, norm_out, norm_row_stride,
+                                       cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, hidden, eps,
+                                       DIT_DTYPE_BF16, stream);
+}
+
+dit_status dit_gated_residual_adaln_ex(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                                       const void* gate, int64_t gate_seq_stride,
+                                       const void* shift, const void* scale, int64_t mod_seq_stride,
+                                       void* res_out, int64_t res_row_stride, void* norm_out,
+                                       int64_t norm_row_stride, const int32_t* cu_seqlens,
+                                       const int32_t* cu_seqlens_padded, int32_t num_seqs,
+                                       int64_t num_rows_padded, int32_t hidden, float eps, int32_t mod_dtype,
+                                       void* stream)
+{
+    if (!known_dtype(mod_dtype))
+        return DIT_ERR_UNSUPPORTED;
+    const bool f32 = mod_dtype == DIT_DTYPE_F32;
     bool empty = false;
     dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
     if (st != DIT_OK)
@@ -220,15 +272,14 @@ dit_status dit_gated_residual_adaln(const void* x, int64_t x_row_stride, const v
         return DIT_ERR_NULL;
     if (!aligned16(x) || !aligned16(y) || !aligned16(gate) || !aligned16(shift) || !aligned16(scale) ||
         !aligned16(res_out) || !aligned16(norm_out) || !mult8(hidden) || !mult8(x_row_stride) ||
-        !mult8(y_row_stride) || !mult8(res_row_stride) || !mult8(norm_row_stride) || !mult8(gate_seq_stride) ||
-        !mult8(mod_seq_stride))
+        !mult8(y_row_stride) || !mult8(res_row_stride) || !mult8(norm_row_stride) ||
+        !mod_stride_ok(gate_seq_stride, f32) || !mod_stride_ok(mod_seq_stride, f32))
         return DIT_ERR_ALIGN;
-    dit::FusedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y),
-                       static_cast<const uint16_t*>(gate), static_cast<const uint16_t*>(shift),
-                       static_cast<const uint16_t*>(scale), static_cast<uint16_t*>(res_out),
-                       static_cast<uint16_t*>(norm_out), x_row_stride, y_row_stride, gate_seq_stride,
-                       mod_seq_stride, res_row_stride, norm_row_stride,
-                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps};
+    dit::FusedParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(y), gate, shift, scale,
+                       static_cast<uint16_t*>(res_out), static_cast<uint16_t*>(norm_out), x_row_stride,
+                       y_row_stride, gate_seq_stride, mod_seq_stride, res_row_stride, norm_row_stride,
+                       packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded), hidden, eps,
+                       f32 ? 1 : 0};
     return from_cuda(dit::launch_gated_residual_adaln(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -185,6 +185,28 @@ __device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) { return __fadd2_rn(a,
 __device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
 __device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) { return __ffma2_rn(a, b, c); }
 
+// Eight consecutive elements, starting at element `elem`, of a per-sequence
+// vector stored as bf16 (F32 false) or fp32 (F32 true), as four fp32 pairs.
+// These vectors are shared by every row of a sequence: read-only path.
+template <bool F32>
+__device__ __forceinline__ void vec8_pairs(const void* base, int64_t elem, f32x2 (&v)[4])
+{
+    if (F32) {
+        const float4* f = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+        const float4 a = __ldg(f), b = __ldg(f + 1);
+        v[0] = make_float2(a.x, a.y);
+        v[1] = make_float2(a.z, a.w);
+        v[2] = make_float2(b.x, b.y);
+        v[3] = make_float2(b.z, b.w);
+    } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem));
+        v[0] = f2_from_bf16x2(u.x);
+        v[1] = f2_from_bf16x2(u.y);
+        v[2] = f2_from_bf16x2(u.z);
+        v[3] = f2_from_bf16x2(u.w);
+    }
+}
+
 // fp32 pair -> bf16x2 word, round to nearest even.
 __device__ __forceinline__ uint32_t f2_to_bf16x2(f32x2 v)
 {

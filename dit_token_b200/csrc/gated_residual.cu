@@ -5,9 +5,10 @@
 //
 // One warp per valid row; each lane streams U 16-byte vectors of x and y per
 // step (all loads of a step are issued before any arithmetic), adds
-// gate * y with one fp32 FMA per element and rounds once.  The gate vector is
-// read through the read-only path: it is shared by every row of a sequence and
-// stays in L1/L2.  HBM traffic: 6 bytes per element (x, y in; out out).
+// gate * y with one fp32 FMA per element and rounds once.  The gate vector
+// (bf16, or fp32 as the modulation head may emit it) is read through the
+// read-only path: it is shared by every row of a sequence and stays in L1/L2.
+// HBM traffic: 6 bytes per element (x, y in; out out).
 #include "common.cuh"
 #include "launch.h"
 
@@ -19,6 +20,7 @@ namespace {
 #endif
 constexpr int kUnroll = DIT_EW_UNROLL;  // 16-byte vectors per lane and input in flight
 
+template <bool F32>
 __global__ void __launch_bounds__(kCtaThreads)
 gated_residual_kernel(const GatedParams p)
 {
@@ -30,33 +32,33 @@ gated_residual_kernel(const GatedParams p)
         return;
     const uint16_t* xr = p.x + (int64_t)s.row * p.x_row_stride;
     const uint16_t* yr = p.y + (int64_t)s.row * p.y_row_stride;
-    const uint16_t* gr = p.gate + (int64_t)s.seq * p.gate_seq_stride;
+    const int64_t goff = (int64_t)s.seq * p.gate_seq_stride;
     uint16_t* orow = p.out + (int64_t)s.row * p.out_row_stride;
     const int nvec = p.hidden / 8;
 
     for (int c0 = 0; c0 < nvec; c0 += kWarp * kUnroll) {
-        uint4 xv[kUnroll], yv[kUnroll], gv[kUnroll];
+        uint4 xv[kUnroll], yv[kUnroll];
+        f32x2 gv[kUnroll][4];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int j = c0 + u * kWarp + lane;
             if (j < nvec) {
                 xv[u] = ld_stream(xr + 8 * j);
                 yv[u] = ld_stream(yr + 8 * j);
-                gv[u] = ld_shared_vec(gr + 8 * j);
+                vec8_pairs<F32>(p.gate, goff + 8 * j, gv[u]);
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int j = c0 + u * kWarp + lane;
             if (j < nvec) {
-                float xf[8], yf[8], gf[8], o[8];
-                unpack8(xv[u], xf);
-                unpack8(yv[u], yf);
-                unpack8(gv[u], gf);
+                const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+                const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
+                uint32_t o[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    o[e] = fmaf(gf[e], yf[e], xf[e]);
-                st_stream(orow + 8 * j, pack8(o));
+                for (int e = 0; e < 4; ++e)
+                    o[e] = f2_to_bf16x2(f2_fma(gv[u][e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
+                st_stream(orow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
             }
         }
     }
@@ -67,7 +69,10 @@ gated_residual_kernel(const GatedParams p)
 cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)((p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta);
-    gated_residual_kernel<<<grid, kCtaThreads, 0, stream>>>(p);
+    if (p.gate_f32)
+        gated_residual_kernel<true><<<grid, kCtaThreads, 0, stream>>>(p);
+    else
+        gated_residual_kernel<false><<<grid, kCtaThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -13,14 +13,15 @@
 //
 // Layout as in adaln_modulate.cu: a team of TEAM warps owns a row and keeps
 // the rounded residual in registers (VPT 16-byte vectors per lane); one-pass
-// moments for the statistics, packed fp32 pairs for the arithmetic.
+// moments for the statistics, packed fp32 pairs for the arithmetic.  gate,
+// shift and scale are bf16, or all three fp32.
 #include "common.cuh"
 #include "launch.h"
 
 namespace dit {
 namespace {
 
-template <int VPT, int TEAM>
+template <int VPT, int TEAM, bool F32>
 __global__ void __launch_bounds__(kCtaThreads, MinCtas<VPT, 2>::value)
 gated_residual_adaln_kernel(const FusedParams p)
 {
@@ -53,20 +54,20 @@ gated_residual_adaln_kernel(const FusedParams p)
             xv[i] = in ? ld_stream(xr + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
             yv[i] = in ? ld_stream(yr + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
         }
-        const uint16_t* gr = p.gate + (int64_t)s.seq * p.gate_seq_stride;
+        const int64_t goff = (int64_t)s.seq * p.gate_seq_stride;
         uint16_t* res = p.res_out + (int64_t)s.row * p.res_row_stride;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int j = i * kTeamThreads + tt;
             if (j < nvec) {
-                const uint4 gv = ld_shared_vec(gr + 8 * j);
+                f32x2 g[4];
+                vec8_pairs<F32>(p.gate, goff + 8 * j, g);
                 const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
                 const uint32_t yw[4] = {yv[i].x, yv[i].y, yv[i].z, yv[i].w};
-                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
                 uint32_t o[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    o[e] = f2_to_bf16x2(f2_fma(f2_from_bf16x2(gw[e]), f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
+                    o[e] = f2_to_bf16x2(f2_fma(g[e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
                 rv[i] = make_uint4(o[0], o[1], o[2], o[3]);
                 st_stream(res + 8 * j, rv[i]);
             } else {
@@ -113,23 +114,21 @@ gated_residual_adaln_kernel(const FusedParams p)
     const f32x2 b2 = f2_make(nb, nb);
     const f32x2 one2 = f2_make(1.f, 1.f);
 
-    const uint16_t* sh = p.shift + (int64_t)s.seq * p.mod_seq_stride;
-    const uint16_t* sc = p.scale + (int64_t)s.seq * p.mod_seq_stride;
+    const int64_t moff = (int64_t)s.seq * p.mod_seq_stride;
     uint16_t* nrow = p.norm_out + (int64_t)s.row * p.norm_row_stride;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
-            const uint4 shv = ld_shared_vec(sh + 8 * j);
-            const uint4 scv = ld_shared_vec(sc + 8 * j);
+            f32x2 hv[4], cv[4];
+            vec8_pairs<F32>(p.shift, moff + 8 * j, hv);
+            vec8_pairs<F32>(p.scale, moff + 8 * j, cv);
             const uint32_t rw[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
-            const uint32_t hw[4] = {shv.x, shv.y, shv.z, shv.w};
-            const uint32_t cw[4] = {scv.x, scv.y, scv.z, scv.w};
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const f32x2 t = f2_fma(f2_from_bf16x2(rw[e]), r2, b2);
-                o[e] = f2_to_bf16x2(f2_fma(t, f2_add(f2_from_bf16x2(cw[e]), one2), f2_from_bf16x2(hw[e])));
+                o[e] = f2_to_bf16x2(f2_fma(t, f2_add(cv[e], one2), hv[e]));
             }
             st_stream(nrow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
         }
@@ -141,7 +140,10 @@ void launch_one(const FusedParams& p, cudaStream_t stream)
 {
     const int rows_per_cta = kWarpsPerCta / TEAM;
     const unsigned grid = (unsigned)((p.pk.num_rows_padded + rows_per_cta - 1) / rows_per_cta);
-    gated_residual_adaln_kernel<VPT, TEAM><<<grid, kCtaThreads, 0, stream>>>(p);
+    if (p.mod_f32)
+        gated_residual_adaln_kernel<VPT, TEAM, true><<<grid, kCtaThreads, 0, stream>>>(p);
+    else
+        gated_residual_adaln_kernel<VPT, TEAM, false><<<grid, kCtaThreads, 0, stream>>>(p);
 }
 
 template <int TEAM>

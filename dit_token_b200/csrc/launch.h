@@ -45,20 +45,21 @@ struct QkParams {
 struct AdalnParams {
     const uint16_t* x;
     uint16_t* out;
-    const uint16_t* shift;
-    const uint16_t* scale;
+    const void* shift;  // bf16 or fp32 (mod_f32)
+    const void* scale;
     int64_t x_row_stride;
     int64_t out_row_stride;
     int64_t mod_seq_stride;
     Packing pk;
     int32_t hidden;
     float eps;
+    int32_t mod_f32;
 };
 
 struct GatedParams {
     const uint16_t* x;
     const uint16_t* y;
-    const uint16_t* gate;
+    const void* gate;  // bf16 or fp32 (gate_f32)
     uint16_t* out;
     int64_t x_row_stride;
     int64_t y_row_stride;
@@ -66,14 +67,15 @@ struct GatedParams {
     int64_t out_row_stride;
     Packing pk;
     int32_t hidden;
+    int32_t gate_f32;
 };
 
 struct FusedParams {
     const uint16_t* x;
     const uint16_t* y;
-    const uint16_t* gate;
-    const uint16_t* shift;
-    const uint16_t* scale;
+    const void* gate;  // gate, shift, scale: bf16 or fp32 (mod_f32)
+    const void* shift;
+    const void* scale;
     uint16_t* res_out;
     uint16_t* norm_out;
     int64_t x_row_stride;
@@ -85,6 +87,7 @@ struct FusedParams {
     Packing pk;
     int32_t hidden;
     float eps;
+    int32_t mod_f32;
 };
 
 struct SwigluParams {

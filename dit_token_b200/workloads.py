@@ -178,10 +178,12 @@ def _threads() -> int:
 
 
 def normal_bf16(shape, seed_seq: np.random.SeedSequence, mean: float = 0.0,
-                std: float = 1.0) -> torch.Tensor:
-    """A CPU bf16 tensor of N(mean, std^2) draws, deterministic in seed_seq."""
+                std: float = 1.0, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """A CPU bf16 tensor of N(mean, std^2) draws, deterministic in seed_seq.
+    With dtype=torch.float32 the same draws are returned unrounded (the bf16
+    tensor is their round-to-nearest-even image)."""
     n = int(math.prod(shape))
-    out = torch.empty(n, dtype=torch.bfloat16)
+    out = torch.empty(n, dtype=dtype)
     nchunks = max(1, -(-n // _CHUNK))
     children = seed_seq.spawn(nchunks)
 
@@ -245,11 +247,12 @@ def qk_inputs(w: Workload) -> dict:
     }
 
 
-def modulation(w: Workload) -> torch.Tensor:
+def modulation(w: Workload, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     """Per-sequence modulation vectors [num_seqs, 6, hidden] ~ N(0, 0.1):
     (shift, scale, gate) of the attention sublayer, then of the MLP sublayer.
-    Operators receive one slice with a sequence stride of 6 * hidden."""
-    return normal_bf16((w.num_seqs, 6, w.hidden), _seed(w, "mod"), std=0.1)
+    Operators receive one slice with a sequence stride of 6 * hidden.  dtype
+    float32 gives the same draws unrounded (a modulation head kept in fp32)."""
+    return normal_bf16((w.num_seqs, 6, w.hidden), _seed(w, "mod"), std=0.1, dtype=dtype)
 
 
 def adaln_inputs(w: Workload) -> dict:

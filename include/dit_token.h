@@ -181,6 +181,44 @@ DIT_API dit_status dit_gated_residual_adaln(const void* x, int64_t x_row_stride,
                                             const int32_t* cu_seqlens_padded, int32_t num_seqs,
                                             int64_t num_rows_padded, int32_t hidden, float eps, void* stream);
 
+/* Element types of the per-sequence modulation vectors (gate, shift, scale)
+ * accepted by the _ex entry points below.  The pages fix no precision for
+ * them; a modulation head may emit them in bf16 or keep them in fp32.  The
+ * activations stay bf16 either way, and every op computes in fp32, so an fp32
+ * vector only removes the rounding of the vector itself. */
+#define DIT_DTYPE_BF16 0
+#define DIT_DTYPE_F32 1
+
+/* dit_adaln_modulate with shift and scale of element type mod_dtype
+ * (DIT_DTYPE_BF16 or DIT_DTYPE_F32).  For fp32 vectors mod_seq_stride must be a
+ * multiple of 4 (16-byte aligned vectors); for bf16 a multiple of 8.  An
+ * unknown mod_dtype returns DIT_ERR_UNSUPPORTED. */
+DIT_API dit_status dit_adaln_modulate_ex(const void* x, int64_t x_row_stride, void* out, int64_t out_row_stride,
+                                         const void* shift, const void* scale, int64_t mod_seq_stride,
+                                         const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                         int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, float eps,
+                                         int32_t mod_dtype, void* stream);
+
+/* dit_gated_residual with a gate of element type gate_dtype (same codes and
+ * stride rule as above). */
+DIT_API dit_status dit_gated_residual_ex(const void* x, int64_t x_row_stride, const void* y, int64_t y_row_stride,
+                                         const void* gate, int64_t gate_seq_stride, void* out,
+                                         int64_t out_row_stride, const int32_t* cu_seqlens,
+                                         const int32_t* cu_seqlens_padded, int32_t num_seqs,
+                                         int64_t num_rows_padded, int32_t hidden, int32_t gate_dtype, void* stream);
+
+/* dit_gated_residual_adaln with gate, shift and scale all of element type
+ * mod_dtype (same codes; gate_seq_stride and mod_seq_stride follow the stride
+ * rule above). */
+DIT_API dit_status dit_gated_residual_adaln_ex(const void* x, int64_t x_row_stride, const void* y,
+                                               int64_t y_row_stride, const void* gate, int64_t gate_seq_stride,
+                                               const void* shift, const void* scale, int64_t mod_seq_stride,
+                                               void* res_out, int64_t res_row_stride, void* norm_out,
+                                               int64_t norm_row_stride, const int32_t* cu_seqlens,
+                                               const int32_t* cu_seqlens_padded, int32_t num_seqs,
+                                               int64_t num_rows_padded, int32_t hidden, float eps,
+                                               int32_t mod_dtype, void* stream);
+
 /* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)).
  *
  * Pages: first page "Key takeaways" bullet 2 and third page "vLLM-Omni 中的

@@ -117,10 +117,17 @@ def oracle_qk(w, inp, rows, rope_mode="interleaved"):
                                   rope_mode=rope_mode)
 
 
+def mod_flat(mod: torch.Tensor) -> np.ndarray:
+    """The [num_seqs, 6, hidden] modulation tensor flattened for the oracle:
+    bf16 bit patterns (uint16) or fp32 values, as the tensor holds them."""
+    if mod.dtype == torch.float32:
+        return np.ascontiguousarray(mod.detach().cpu().numpy().reshape(-1))
+    return np.ascontiguousarray(tbits(mod).reshape(-1))
+
+
 def oracle_adaln(w, inp, rows):
     x = tbits(W.rows_view(inp["x"]))
-    mod = tbits(inp["mod"]).reshape(w.num_seqs, 6 * w.hidden)
-    flat = np.ascontiguousarray(mod.reshape(-1))
+    flat = mod_flat(inp["mod"])
     return oracle.adaln_modulate(x, flat, flat[w.hidden:], w.cu_seqlens, w.cu_seqlens_padded,
                                  hidden=w.hidden, eps=w.eps, mod_seq_stride=6 * w.hidden, rows=rows)
 
@@ -128,7 +135,7 @@ def oracle_adaln(w, inp, rows):
 def oracle_residual(w, inp, rows):
     x = tbits(W.rows_view(inp["x"]))
     y = tbits(W.rows_view(inp["y"]))
-    flat = np.ascontiguousarray(tbits(inp["mod"]).reshape(-1))
+    flat = mod_flat(inp["mod"])
     return oracle.gated_residual(x, y, flat[2 * w.hidden:], w.cu_seqlens, w.cu_seqlens_padded,
                                  hidden=w.hidden, gate_seq_stride=6 * w.hidden, rows=rows)
 
@@ -136,7 +143,7 @@ def oracle_residual(w, inp, rows):
 def oracle_fused(w, inp, rows):
     x = tbits(W.rows_view(inp["x"]))
     y = tbits(W.rows_view(inp["y"]))
-    flat = np.ascontiguousarray(tbits(inp["mod"]).reshape(-1))
+    flat = mod_flat(inp["mod"])
     C = w.hidden
     return oracle.gated_residual_adaln(x, y, flat[2 * C:], flat[3 * C:], flat[4 * C:], w.cu_seqlens,
                                        w.cu_seqlens_padded, hidden=C, eps=w.eps, gate_seq_stride=6 * C,

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 11, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(L, n), n
     assert L.dit_abi_version() == 1
@@ -145,6 +145,32 @@ def test_fused_residual_adaln_argument_checks(L):
     assert call(B=0, x=None, n=None) == OK
 
 
+def test_modulation_dtype_entries(L):
+    """The _ex entries take a dtype code (0 bf16, 1 fp32); fp32 vectors need a
+    sequence stride that is a multiple of 4, bf16 ones a multiple of 8."""
+    def ada(dt, ms=64):
+        return L.dit_adaln_modulate_ex(P, 64, P, 64, P, P, ms, P, P, 0, 4, 64, 1e-6, dt, None)
+    def res(dt, gs=64, B=0):
+        return L.dit_gated_residual_ex(P, 64, P, 64, P, gs, P, 64, P, P, B, 4, 64, dt, None)
+    def fused(dt, gs=64, ms=64, g=P):
+        return L.dit_gated_residual_adaln_ex(P, 64, P, 64, g, gs, P, P, ms, P, 64, P, 64, P, P, 0, 4, 64, 1e-6,
+                                             dt, None)
+    for f in (ada, res, fused):
+        assert f(2) == UNSUP and f(-1) == UNSUP
+        assert f(0) == OK and f(1) == OK     # empty batches: checks only, no launch
+    assert ada(1, ms=68) == OK and ada(0, ms=68) == OK            # empty: strides unchecked
+    assert fused(1, g=None) == OK                                  # empty batch: no pointer needed
+    # non-empty calls stop at the alignment check, before any launch
+    assert L.dit_adaln_modulate_ex(P, 64, P, 64, P, P, 68, P, P, 1, 4, 64, 1e-6, 0, None) == ALIGN
+    assert L.dit_adaln_modulate_ex(P, 64, P, 64, P, P, 66, P, P, 1, 4, 64, 1e-6, 1, None) == ALIGN
+    assert L.dit_gated_residual_ex(P, 64, P, 64, P, 12, P, 64, P, P, 2, 4, 64, 0, None) == ALIGN
+    assert L.dit_gated_residual_ex(P, 64, P, 64, P, 10, P, 64, P, P, 2, 4, 64, 1, None) == ALIGN
+    assert L.dit_gated_residual_adaln_ex(P, 64, P, 64, P, 64, P, P, 66, P, 64, P, 64, P, P, 1, 4, 64, 1e-6, 1,
+                                         None) == ALIGN
+    assert L.dit_gated_residual_adaln_ex(P, 64, P, 64, None, 64, P, P, 64, P, 64, P, 64, P, P, 1, 4, 64, 1e-6,
+                                         1, None) == NULL
+
+
 def test_frames_argument_checks(L):
     assert L.dit_frames_to_u8(P, 1, 3, 2, 4, 16, 2, P, None) == UNSUP
     assert L.dit_frames_to_u8(P, 1, -3, 2, 4, 16, 0, P, None) == SHAPE
@@ -171,3 +197,7 @@ def test_binding_rejects_cpu_tensors_before_the_library():
         dit.dit_gated_residual(x, x, torch.zeros(1, 8, dtype=torch.bfloat16), cs, cs)
     with pytest.raises(TypeError):
         dit.dit_swiglu(x.float(), x.float(), cs, cs)
+    with pytest.raises(TypeError):   # fp16 modulation vectors are not accepted
+        dit._seq_vectors(torch.zeros(1, 8, dtype=torch.float16), 8, "gate")
+    with pytest.raises(TypeError):   # mixed bf16 / fp32 vectors in one call
+        dit._one_dtype((0, 1, 0), "gate, shift and scale")

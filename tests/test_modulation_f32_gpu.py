@@ -1,0 +1,106 @@
+"""fp32 per-sequence modulation vectors (gate, shift, scale) on the GPU, through
+the _ex entry points, against the oracle's fp32 path.
+
+The activations stay bf16; the vectors are the unrounded N(0, 0.1) draws whose
+rounding is the bf16 modulation of the same workload.  Three checks:
+parity with the oracle at every adaLN team shape and on many short sequences
+(more sequences per CTA than the adaLN kernel stages in shared memory); bit
+equality with the bf16 path when the fp32 vectors hold bf16 values; and
+sampled rows of the full batched-varlen workload.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dit_token_b200 as dit
+from dit_token_b200 import workloads as W
+import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from dit_token_b200 import build
+    build.build()
+
+
+def with_f32_mod(w, inp):
+    out = dict(inp)
+    out["mod"] = W.modulation(w, torch.float32)
+    return out
+
+
+def check_three_ops(w, rows, tag):
+    keep = P.untouched_rows(w)
+    inp = with_f32_mod(w, W.adaln_inputs(w))
+    out = P.gpu_adaln(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_adaln(w, inp, rows)[rows], f"{tag} adaln f32")
+    P.assert_untouched(out, inp["out"], keep, f"{tag} adaln f32")
+    inp = with_f32_mod(w, W.residual_inputs(w))
+    out = P.gpu_residual(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_residual(w, inp, rows)[rows], f"{tag} residual f32")
+    P.assert_untouched(out, inp["out"], keep, f"{tag} residual f32")
+    res, norm = P.gpu_fused(w, inp)
+    r_ref, n_ref = P.oracle_fused(w, inp, rows)
+    P.assert_close(P.gather_rows(res, rows), r_ref[rows], f"{tag} fused residual f32")
+    P.assert_close(P.gather_rows(norm, rows), n_ref[rows], f"{tag} fused norm f32")
+    P.assert_untouched(res, inp["out"], keep, f"{tag} fused res f32")
+    P.assert_untouched(norm, inp["out"], keep, f"{tag} fused norm f32")
+    # the fused residual is the separate residual kernel's, bit for bit
+    assert torch.equal(res.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("hidden", [8, 264, 2048, 3072, 5120, 6152, 8192, 16384])
+def test_f32_modulation_every_team_shape(hidden):
+    w = W.custom("mod32", (13, 6), (16, 8), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=hidden + 1)
+    check_three_ops(w, w.valid_rows(), f"hidden {hidden}")
+
+
+def test_f32_modulation_many_short_sequences():
+    rng = np.random.default_rng(11)
+    lengths = rng.integers(0, 7, 400)
+    padded = [int(L) + int(rng.integers(0, 3)) for L in lengths]
+    w = W.custom("mod32many", lengths, padded, hidden=1024, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=4)
+    check_three_ops(w, w.valid_rows(), "many")
+
+
+@pytest.mark.parametrize("hidden", [264, 5120, 8192])
+def test_bf16_valued_f32_vectors_match_the_bf16_path_bitwise(hidden):
+    w = W.custom("same", (37, 5, 90), (40, 8, 96), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=7)
+    cs, cp, _ = P.device_packing(w)
+    inp = W.residual_inputs(w)
+    x, y = W.rows_view(inp["x"].cuda()), W.rows_view(inp["y"].cuda())
+    m16 = inp["mod"].cuda()
+    m32 = m16.float()
+    a = dit.dit_adaln_modulate(x, m16[:, 0], m16[:, 1], cs, cp, eps=w.eps)
+    b = dit.dit_adaln_modulate(x, m32[:, 0], m32[:, 1], cs, cp, eps=w.eps)
+    rows = torch.from_numpy(w.valid_rows()).cuda()
+    assert torch.equal(a[rows].view(torch.int16), b[rows].view(torch.int16))
+    a = dit.dit_gated_residual(x, y, m16[:, 2], cs, cp)
+    b = dit.dit_gated_residual(x, y, m32[:, 2], cs, cp)
+    assert torch.equal(a[rows].view(torch.int16), b[rows].view(torch.int16))
+    ra, na = dit.dit_gated_residual_adaln(x, y, m16[:, 2], m16[:, 3], m16[:, 4], cs, cp, eps=w.eps)
+    rb, nb = dit.dit_gated_residual_adaln(x, y, m32[:, 2], m32[:, 3], m32[:, 4], cs, cp, eps=w.eps)
+    assert torch.equal(ra[rows].view(torch.int16), rb[rows].view(torch.int16))
+    assert torch.equal(na[rows].view(torch.int16), nb[rows].view(torch.int16))
+
+
+def test_f32_modulation_batched_varlen_sampled():
+    w = W.workload("batched_varlen")
+    check_three_ops(w, W.sample_rows(w, per_seq=32), "batched_varlen")
+
+
+def test_mixed_dtypes_are_rejected():
+    w = W.custom("mix", (5,), (8,), hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=8)
+    cs, cp, _ = P.device_packing(w)
+    x = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    g16 = torch.zeros(1, 64, dtype=torch.bfloat16, device="cuda")
+    g32 = torch.zeros(1, 64, dtype=torch.float32, device="cuda")
+    with pytest.raises(TypeError):
+        dit.dit_adaln_modulate(x, g16, g32, cs, cp)
+    with pytest.raises(TypeError):
+        dit.dit_gated_residual_adaln(x, x, g32, g16, g16, cs, cp)
