@@ -57,6 +57,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_gated_residual_adaln_ex.argtypes = [
             u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i32p, i32, i64, i32, f64,
             u16p, i64, u16p, i64, f64p, i64p, i64]
+        L.oracle_adaln_modulate_av.argtypes = [
+            u16p, i64, vp, vp, i64, i32, i32p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
+        L.oracle_gated_residual_av.argtypes = [
+            u16p, i64, u16p, i64, vp, i64, i32, i32p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p,
+            i64]
+        L.oracle_gated_residual_adaln_av.argtypes = [
+            u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i64, i64, i32p, i32p, i32, i64, i32, f64,
+            u16p, i64, u16p, i64, f64p, i64p, i64]
         L.oracle_swiglu.argtypes = [
             u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
         L.oracle_frames_to_u8.argtypes = [ctypes.POINTER(ctypes.c_float), i64, i64, i64, i64, i64, i32,
@@ -65,6 +73,7 @@ def lib() -> ctypes.CDLL:
                      "oracle_frames_to_u8",
                      "oracle_gated_residual", "oracle_gated_residual_adaln", "oracle_swiglu",
                      "oracle_adaln_modulate_ex", "oracle_gated_residual_ex", "oracle_gated_residual_adaln_ex",
+                     "oracle_adaln_modulate_av", "oracle_gated_residual_av", "oracle_gated_residual_adaln_av",
                      "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -195,13 +204,20 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
     return q_out, k_out
 
 
+def _grid(rope_grid):
+    return None if rope_grid is None else np.ascontiguousarray(np.asarray(rope_grid, dtype=np.int32))
+
+
 def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
                    mod_seq_stride=None, x_row_stride=None, rows=None, out_init=None,
-                   want_f64=False, out=None):
+                   want_f64=False, out=None, rope_grid=None, audio_offset=0):
     """out = LayerNorm(x) * (1 + scale_b) + shift_b on valid rows.
 
-    shift, scale: uint16 arrays [num_seqs, ...] read with mod_seq_stride
-    elements between sequences (default: hidden)."""
+    shift, scale: uint16 (bf16 bits) or float32 arrays [num_seqs, ...] read
+    with mod_seq_stride elements between sequences (default: hidden).
+    Per-stream vectors: with rope_grid [num_seqs][3] given, the audio rows of
+    sequence b (local index >= T*H*W) read their vectors audio_offset
+    elements after the video rows' ones."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
@@ -215,8 +231,9 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
         raise TypeError("shift and scale must have the same dtype")
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_adaln_modulate_ex(
-        _ptr(x, ctypes.c_uint16), xs, _vptr(sh), _vptr(sc), mss, f1,
+    grid = _grid(rope_grid)
+    rc = lib().oracle_adaln_modulate_av(
+        _ptr(x, ctypes.c_uint16), xs, _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32), audio_offset,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "adaln_modulate")
@@ -225,8 +242,9 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
 
 def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_seq_stride=None,
                    x_row_stride=None, y_row_stride=None, rows=None, out_init=None,
-                   want_f64=False, out=None):
-    """out = x + gate_b * y on valid rows."""
+                   want_f64=False, out=None, rope_grid=None, audio_offset=0):
+    """out = x + gate_b * y on valid rows (per-stream gates as in
+    adaln_modulate)."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
@@ -238,9 +256,10 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
     g, gf = _mod(gate)
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_gated_residual_ex(
+    grid = _grid(rope_grid)
+    rc = lib().oracle_gated_residual_av(
         _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss, gf,
-        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
+        _ptr(grid, ctypes.c_int32), audio_offset, _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "gated_residual")
     return (out, o64) if want_f64 else out
@@ -249,9 +268,11 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
 def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
                         gate_seq_stride=None, mod_seq_stride=None, x_row_stride=None, y_row_stride=None,
                         rows=None, res_init=None, norm_init=None, want_f64=False, res_out=None,
-                        norm_out=None):
+                        norm_out=None, rope_grid=None, gate_audio_offset=0, mod_audio_offset=0):
     """res = x + gate_b * y (bf16), norm = LN(res) * (1 + scale_b) + shift_b on
-    valid rows.  Returns (res, norm) or, with want_f64, (res, norm, norm_f64)."""
+    valid rows (per-stream vectors as in adaln_modulate, with one audio
+    offset for the gate and one for shift/scale).  Returns (res, norm) or,
+    with want_f64, (res, norm, norm_f64)."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
@@ -270,9 +291,10 @@ def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    rc = lib().oracle_gated_residual_adaln_ex(
+    grid = _grid(rope_grid)
+    rc = lib().oracle_gated_residual_adaln_av(
         _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss,
-        _vptr(sh), _vptr(sc), mss, f1,
+        _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32), gate_audio_offset, mod_audio_offset,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(res_out, ctypes.c_uint16), xs, _ptr(norm_out, ctypes.c_uint16), xs, _ptr(n64, ctypes.c_double),
         _ptr(r, ctypes.c_int64), nr)

@@ -79,6 +79,23 @@ static double ldm(const void* base, int64_t idx, int f32)
 
 /* -------------------------------------------------------- packed rows */
 
+/* Offset of the per-sequence vectors that valid row r of sequence b uses.
+ * One vector set per sequence: b * seq_stride.  With per-stream vectors
+ * (rope_grid != NULL) the joint audio-video sequence holds its T*H*W video
+ * rows first and its audio rows after them; video rows use the set at
+ * b * seq_stride, audio rows the set audio_offset elements further on. */
+static int64_t vec_offset(int32_t b, int64_t r, int64_t seq_stride, const int32_t* rope_grid,
+                          int64_t audio_offset)
+{
+    int64_t off = (int64_t)b * seq_stride;
+    if (rope_grid) {
+        int64_t thw = (int64_t)rope_grid[3 * b] * rope_grid[3 * b + 1] * rope_grid[3 * b + 2];
+        if (r >= thw)
+            off += audio_offset;
+    }
+    return off;
+}
+
 /* The padded buffer holds num_seqs sequences; sequence b owns padded rows
  * [cu_seqlens_padded[b], cu_seqlens_padded[b+1]) and its first
  * cu_seqlens[b+1] - cu_seqlens[b] rows are valid (the rest is structural
@@ -304,6 +321,20 @@ int oracle_adaln_modulate_ex(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_adaln_modulate_av(x, x_row_stride, shift, scale, mod_seq_stride, mod_f32, NULL, 0, cu_seqlens,
+                                    cu_seqlens_padded, num_seqs, num_rows_padded, hidden, eps, out,
+                                    out_row_stride, out_f64, rows, num_rows);
+}
+
+int oracle_adaln_modulate_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!x || !shift || !scale || !out || hidden <= 0)
         return -1;
     if (x_row_stride < hidden || out_row_stride < hidden || mod_seq_stride < 0)
@@ -321,7 +352,7 @@ int oracle_adaln_modulate_ex(
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
         const uint16_t* xr = x + row * x_row_stride;
-        const int64_t mb = (int64_t)b * mod_seq_stride;
+        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, audio_offset);
         /* LayerNorm without affine: mean, then the biased variance about it. */
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
@@ -367,6 +398,21 @@ int oracle_gated_residual_ex(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_gated_residual_av(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, gate_f32, NULL, 0,
+                                    cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, hidden, out,
+                                    out_row_stride, out_f64, rows, num_rows);
+}
+
+int oracle_gated_residual_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
+    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!x || !y || !gate || !out || hidden <= 0)
         return -1;
     if (x_row_stride < hidden || y_row_stride < hidden || out_row_stride < hidden || gate_seq_stride < 0)
@@ -383,7 +429,7 @@ int oracle_gated_residual_ex(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const int64_t gb = (int64_t)b * gate_seq_stride;
+        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, audio_offset);
         for (int32_t c = 0; c < hidden; ++c) {
             double v = ld(&x[row * x_row_stride + c]) + ldm(gate, gb + c, gate_f32) * ld(&y[row * y_row_stride + c]);
             put(out, out_f64, row * out_row_stride + c, v);
@@ -428,6 +474,24 @@ int oracle_gated_residual_adaln_ex(
     uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_gated_residual_adaln_av(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, shift, scale,
+                                          mod_seq_stride, mod_f32, NULL, 0, 0, cu_seqlens, cu_seqlens_padded,
+                                          num_seqs, num_rows_padded, hidden, eps, res_out, res_row_stride,
+                                          norm_out, norm_row_stride, norm_out_f64, rows, num_rows);
+}
+
+int oracle_gated_residual_adaln_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* rope_grid, int64_t gate_audio_offset, int64_t mod_audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!x || !y || !gate || !shift || !scale || !res_out || !norm_out || hidden <= 0)
         return -1;
     if (x_row_stride < hidden || y_row_stride < hidden || res_row_stride < hidden || norm_row_stride < hidden ||
@@ -445,7 +509,7 @@ int oracle_gated_residual_adaln_ex(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const int64_t gb = (int64_t)b * gate_seq_stride;
+        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, gate_audio_offset);
         uint16_t* rr = res_out + row * res_row_stride;
         /* step 1: residual update, stored as bf16 */
         for (int32_t c = 0; c < hidden; ++c) {
@@ -453,7 +517,7 @@ int oracle_gated_residual_adaln_ex(
             rr[c] = oracle_f64_to_bf16(v);
         }
         /* step 2: adaLN of the stored residual */
-        const int64_t mb = (int64_t)b * mod_seq_stride;
+        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, mod_audio_offset);
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
             mean += ld(&rr[c]);

@@ -153,6 +153,43 @@ int oracle_gated_residual_adaln_ex(
     uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
     const int64_t* rows, int64_t num_rows);
 
+/* Per-stream modulation of the joint audio-video sequence (the pages pack
+ * the audio and video tokens of a request into one sequence, "Why Real-Time
+ * MiniMax H3 Serving Requires More Than a Faster DiT", "Key takeaways",
+ * bullet 1; they do not say whether the two streams share modulation
+ * vectors).  Sequence b holds rope_grid[b] = (T, H, W): its first T*H*W valid
+ * rows are video and use the vectors at b * stride; the remaining valid rows
+ * are audio and use the vectors audio_offset elements further on.  With
+ * rope_grid NULL every row uses b * stride (the _ex functions). */
+int oracle_adaln_modulate_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows);
+int oracle_gated_residual_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
+    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
+    uint16_t* out, int64_t out_row_stride, double* out_f64,
+    const int64_t* rows, int64_t num_rows);
+int oracle_gated_residual_adaln_av(
+    const uint16_t* x, int64_t x_row_stride,
+    const uint16_t* y, int64_t y_row_stride,
+    const void* gate, int64_t gate_seq_stride,
+    const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
+    const int32_t* rope_grid, int64_t gate_audio_offset, int64_t mod_audio_offset,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
+    uint16_t* res_out, int64_t res_row_stride,
+    uint16_t* norm_out, int64_t norm_row_stride, double* norm_out_f64,
+    const int64_t* rows, int64_t num_rows);
+
 /* SwiGLU activation: out = silu(a) * b, silu(a) = a / (1 + exp(-a)). */
 int oracle_swiglu(
     const uint16_t* a, int64_t a_row_stride,

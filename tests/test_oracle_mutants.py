@@ -18,7 +18,7 @@ SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
         "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py",
         "tests/test_oracle_frames.py", "tests/test_oracle_rope_modes.py",
-        "tests/test_oracle_modulation_f32.py"]
+        "tests/test_oracle_modulation_f32.py", "tests/test_oracle_av_modulation.py"]
 
 # (name, original text, planted mistake)
 MUTANTS = [
@@ -44,7 +44,9 @@ MUTANTS = [
      "ld(&y[row * y_row_stride + c])"),
     ("fused_gate_dropped", "ldm(gate, gb + c, mod_f32) * ld(&y[row * y_row_stride + c])",
      "ld(&y[row * y_row_stride + c])"),
-    ("gate_not_per_sequence", "const int64_t gb = (int64_t)b * gate_seq_stride;", "const int64_t gb = 0;"),
+    ("vectors_not_per_sequence", "int64_t off = (int64_t)b * seq_stride;", "int64_t off = 0;"),
+    ("audio_split_off_by_one", "if (r >= thw)\n            off += audio_offset;", "if (r > thw)\n            off += audio_offset;"),
+    ("audio_vectors_ignored", "off += audio_offset;", "off += 0;"),
     ("silu_sign", "exp(-av)", "exp(av)"),
     ("swiglu_operands_transposed", "double silu = av / (1.0 + exp(-av));\n            put(out, out_f64, row * out_row_stride + c, silu * bv);",
      "double silu = bv / (1.0 + exp(-bv));\n            put(out, out_f64, row * out_row_stride + c, silu * av);"),
