@@ -629,6 +629,84 @@ def run_table(args):
           f"{100 * gbs / 8000:.1f} | {100 * gbs / peak:.1f} |", flush=True)
 
 
+def run_variants(args):
+    """Markdown table of the operator variants (fp32 and per-stream modulation
+    vectors, rotary layouts, grouped K heads, head_dim 256) on the batched
+    varlen and long video workloads, timed like --table (L2 evicted before
+    every launch, median of --steps launches)."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from dit_token_b200 import build
+    build.build()
+    import dit_token_b200 as dit
+    peak, kind = measured_peak()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    rv = W.rows_view
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.fill_(1)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(device)
+        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3  # us
+
+    def row(wname, op, variant, us, nbytes, tokens):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        print(f"| {wname} | {op} | {variant} | {us:.1f} | {tokens / (us * 1e-6):.3g} | {gbs:.0f} | "
+              f"{100 * gbs / peak:.1f} |", flush=True)
+
+    print(f"| workload | op | variant | GPU us | tokens/s | GB/s | % of {kind} {peak:.0f} GB/s |")
+    print("|---|---|---|---|---|---|---|")
+    for name in ("batched_varlen", "long_video"):
+        w = W.workload(name, args.seed)
+        C, B, n = w.hidden, w.num_seqs, w.num_valid
+        step = Step(w, host_inputs(w), device)
+        m32 = W.modulation(w, torch.float32).to(device)
+        cs2, cp2 = dit.dit_av_stream_seqlens(step.cs, step.cp, step.grid)
+        mav = W.modulation_av(w).to(device).view(2 * B, 6, C)
+        mods = {"bf16 vectors": (step.mod, step.cs, step.cp), "fp32 vectors": (m32, step.cs, step.cp),
+                "per-stream bf16 vectors": (mav, cs2, cp2)}
+        for variant, (m, cs, cp) in mods.items():
+            row(name, "adaln_modulate", variant, timed(lambda: dit.dit_adaln_modulate(
+                rv(step.ax), m[:, 0], m[:, 1], cs, cp, out=rv(step.aout), eps=w.eps)), 4 * C * n, n)
+            row(name, "gated_residual", variant, timed(lambda: dit.dit_gated_residual(
+                rv(step.rx), rv(step.ry), m[:, 2], cs, cp, out=rv(step.rout))), 6 * C * n, n)
+            row(name, "gated_residual_adaln", variant, timed(lambda: dit.dit_gated_residual_adaln(
+                rv(step.rx), rv(step.ry), m[:, 2], m[:, 3], m[:, 4], cs, cp, res_out=rv(step.rout),
+                norm_out=rv(step.aout), eps=w.eps)), 8 * C * n, n)
+        row(name, "av_stream_seqlens", f"{B} requests", timed(lambda: dit.dit_av_stream_seqlens(
+            step.cs, step.cp, step.grid, out=(cs2, cp2))), 0, n)
+        for mode in ("interleaved", "half", "none"):
+            row(name, "qk_rmsnorm_rope", f"{mode} pairs, {w.num_q_heads}x{w.head_dim}",
+                timed(lambda: dit.dit_qk_rmsnorm_rope(
+                    rv(step.q), rv(step.k), step.wq, step.wk, step.cs, step.cp, num_q_heads=w.num_q_heads,
+                    num_k_heads=w.num_k_heads, head_dim=w.head_dim, rope_grid=step.grid, sections=w.sections,
+                    rope_theta=w.rope_theta, eps=w.eps, rope_mode=mode)), 8 * C * n, n)
+        # grouped K heads (a fifth of the q heads), and head_dim 256 over the same q and k widths
+        hk = max(1, w.num_q_heads // 5)
+        kq = rv(step.k)[:, : hk * w.head_dim]
+        row(name, "qk_rmsnorm_rope", f"GQA {w.num_q_heads}q/{hk}k x{w.head_dim}", timed(
+            lambda: dit.dit_qk_rmsnorm_rope(
+                rv(step.q), kq, step.wq, step.wk, step.cs, step.cp, num_q_heads=w.num_q_heads, num_k_heads=hk,
+                head_dim=w.head_dim, rope_grid=step.grid, sections=w.sections, rope_theta=w.rope_theta,
+                eps=w.eps)), 4 * (w.num_q_heads + hk) * w.head_dim * n, n)
+        w256 = torch.ones(256, dtype=torch.bfloat16, device=device)
+        for mode, sec in (("half", (88, 84, 84)), ("none", (0, 0, 0))):
+            row(name, "qk_rmsnorm_rope", f"{mode} pairs, {C // 256}x256", timed(
+                lambda: dit.dit_qk_rmsnorm_rope(
+                    rv(step.q), rv(step.k), w256, w256, step.cs, step.cp, num_q_heads=C // 256,
+                    num_k_heads=C // 256, head_dim=256, rope_grid=step.grid, sections=sec,
+                    rope_theta=w.rope_theta, eps=w.eps, rope_mode=mode)), 8 * C * n, n)
+        del step, mods, m32, mav
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -645,6 +723,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true",
                     help="print a per-op markdown table over every workload instead of the JSON line")
+    ap.add_argument("--variants", action="store_true",
+                    help="print a markdown table of the operator variants instead of the JSON line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -654,6 +734,8 @@ def main(argv=None):
             ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
     if args.table:
         run_table(args)
+    elif args.variants:
+        run_variants(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

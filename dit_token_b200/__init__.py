@@ -69,6 +69,7 @@ _SIGNATURES = {
     "dit_gated_residual_adaln_ex": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _I64, _VP, _I64,
                                     _VP, _VP, _I32, _I64, _I32, _F32, _I32, _VP],
     "dit_validate_seqlens": [_VP, _VP, _I32, _I64, _VP, _VP],
+    "dit_av_stream_seqlens": [_VP, _VP, _VP, _I32, _VP, _VP, _VP],
     "dit_frames_to_u8": [_VP, _I64, _I64, _I64, _I64, _I64, _I32, _VP, _VP],
     "dit_status_string": [_I32],
     "dit_last_cuda_error": [],
@@ -323,6 +324,29 @@ def dit_validate_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tens
         flag = torch.empty(2, dtype=torch.int32, device=cu_seqlens.device)
     _call("dit_validate_seqlens", cs, cp, B, int(num_rows_padded), flag.data_ptr(), _stream(stream))
     return flag
+
+
+def dit_av_stream_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, rope_grid: torch.Tensor,
+                          *, out: Optional[tuple] = None, stream=None) -> tuple:
+    """Per-stream descriptor of joint audio-video sequences: sequence b becomes
+    sequences 2b (its T*H*W video rows) and 2b + 1 (its audio rows and
+    padding).  Returns (cu_seqlens_av, cu_seqlens_padded_av), int32
+    [2 * num_seqs + 1] on the device.  Pass them to the modulated ops with
+    vectors laid out [num_seqs, 2, ...] viewed as [2 * num_seqs, ...], e.g. for
+    mod [B, 2, 6, C]: shift = mod.view(2 * B, 6, C)[:, 0]."""
+    cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
+    if rope_grid.dtype != torch.int32 or not rope_grid.is_cuda or not rope_grid.is_contiguous() or \
+            tuple(rope_grid.shape) != (B, 3):
+        raise TypeError("rope_grid: expected a contiguous int32 CUDA tensor [num_seqs, 3]")
+    if out is None:
+        out = (torch.empty(2 * B + 1, dtype=torch.int32, device=cu_seqlens.device),
+               torch.empty(2 * B + 1, dtype=torch.int32, device=cu_seqlens.device))
+    for t in out:
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != 2 * B + 1:
+            raise TypeError(f"out: expected two contiguous int32 CUDA vectors of {2 * B + 1} entries")
+    _call("dit_av_stream_seqlens", cs, cp, rope_grid.data_ptr(), B, out[0].data_ptr(), out[1].data_ptr(),
+          _stream(stream))
+    return out
 
 
 def check_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, num_rows_padded: int,

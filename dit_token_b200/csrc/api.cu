@@ -341,6 +341,25 @@ dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seq
     return from_cuda(dit::launch_validate_seqlens(pk, num_rows_padded, flag, static_cast<cudaStream_t>(stream)));
 }
 
+dit_status dit_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                 const int32_t* rope_grid, int32_t num_seqs, int32_t* out_cu_seqlens,
+                                 int32_t* out_cu_seqlens_padded, void* stream)
+{
+    if (num_seqs < 0 || num_seqs > (INT32_MAX - 1) / 2)
+        return DIT_ERR_SHAPE;
+    if (!cu_seqlens || !cu_seqlens_padded || !out_cu_seqlens || !out_cu_seqlens_padded ||
+        (num_seqs > 0 && !rope_grid))
+        return DIT_ERR_NULL;
+    const uintptr_t any = reinterpret_cast<uintptr_t>(cu_seqlens) | reinterpret_cast<uintptr_t>(cu_seqlens_padded) |
+                          reinterpret_cast<uintptr_t>(rope_grid) | reinterpret_cast<uintptr_t>(out_cu_seqlens) |
+                          reinterpret_cast<uintptr_t>(out_cu_seqlens_padded);
+    if (any & 3u)
+        return DIT_ERR_ALIGN;
+    return from_cuda(dit::launch_av_stream_seqlens(cu_seqlens, cu_seqlens_padded, rope_grid, num_seqs,
+                                                   out_cu_seqlens, out_cu_seqlens_padded,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 const char* dit_status_string(dit_status s)
 {
     switch (s) {

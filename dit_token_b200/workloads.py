@@ -46,7 +46,7 @@ _CHUNK = 1 << 22
 # Child-seed slots: one per tensor, so building one operator's inputs never
 # shifts another's values.
 _SLOT = {"q": 0, "k": 1, "q_weight": 2, "k_weight": 3, "adaln_x": 4, "mod": 5,
-         "res_x": 6, "res_y": 7, "ab": 8}
+         "res_x": 6, "res_y": 7, "ab": 8, "mod_av": 9}
 
 WORKLOAD_NAMES = ("tiny", "single_stream", "video", "long_video", "batched_varlen")
 
@@ -253,6 +253,12 @@ def modulation(w: Workload, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor
     Operators receive one slice with a sequence stride of 6 * hidden.  dtype
     float32 gives the same draws unrounded (a modulation head kept in fp32)."""
     return normal_bf16((w.num_seqs, 6, w.hidden), _seed(w, "mod"), std=0.1, dtype=dtype)
+
+
+def modulation_av(w: Workload, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """Per-stream modulation vectors [num_seqs, 2, 6, hidden] ~ N(0, 0.1):
+    stream 0 for a request's video rows, stream 1 for its audio rows."""
+    return normal_bf16((w.num_seqs, 2, 6, w.hidden), _seed(w, "mod_av"), std=0.1, dtype=dtype)
 
 
 def adaln_inputs(w: Workload) -> dict:

@@ -266,6 +266,31 @@ DIT_API dit_status dit_frames_to_u8(const float* x, int64_t batch, int64_t chann
 DIT_API dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
                                 int32_t num_seqs, int64_t num_rows_padded, int32_t* flag, void* stream);
 
+/* Per-stream packing descriptor of joint audio-video sequences.
+ *
+ * Pages: first page "Key takeaways" bullet 1 (a request's audio and video
+ * tokens are packed into one sequence); whether the two streams share
+ * modulation vectors is left open, and this call lets them differ.
+ * Sequence b of (cu_seqlens, cu_seqlens_padded) holds v_b = clamp(T*H*W, 0,
+ * min(L_b, padded_b)) video rows (rope_grid[b] = (T, H, W)) and then its audio
+ * rows and suffix padding.  The output describes 2*num_seqs sequences:
+ *   2b     the video rows of b:       valid v_b, padded v_b
+ *   2b + 1 the audio rows of b:       valid L_b - v_b, padded padded_b - v_b
+ * over the same buffer rows.  Passing it to dit_adaln_modulate(_ex),
+ * dit_gated_residual(_ex) or dit_gated_residual_adaln(_ex) with vectors laid out
+ * [num_seqs][2 streams][...] (sequence stride of the output = the stride
+ * between the two streams' sets) applies the video set to video rows and the
+ * audio set to audio rows.  RoPE keeps the original descriptor (positions are
+ * per request).
+ *
+ * cu_seqlens, cu_seqlens_padded  device int32 [num_seqs + 1]
+ * rope_grid                      device int32 [num_seqs][3] (may be NULL only if num_seqs == 0)
+ * out_cu_seqlens, out_cu_seqlens_padded  device int32 [2 * num_seqs + 1], written
+ * One small kernel on `stream`; no synchronization.  Entries 0 are copied. */
+DIT_API dit_status dit_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                         const int32_t* rope_grid, int32_t num_seqs, int32_t* out_cu_seqlens,
+                                         int32_t* out_cu_seqlens_padded, void* stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 DIT_API const char* dit_status_string(dit_status s);
 

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 14, names
+    assert len(names) == 15, names
     for n in names:
         assert hasattr(L, n), n
     assert L.dit_abi_version() == 1
@@ -169,6 +169,16 @@ def test_modulation_dtype_entries(L):
                                          None) == ALIGN
     assert L.dit_gated_residual_adaln_ex(P, 64, P, 64, None, 64, P, P, 64, P, 64, P, 64, P, P, 1, 4, 64, 1e-6,
                                          1, None) == NULL
+
+
+def test_av_stream_seqlens_argument_checks(L):
+    f = L.dit_av_stream_seqlens
+    assert f(P, P, P, -1, P, P, None) == SHAPE
+    assert f(P, P, P, 1 << 30, P, P, None) == SHAPE
+    assert f(None, P, P, 2, P, P, None) == NULL
+    assert f(P, P, None, 2, P, P, None) == NULL        # the split needs the grid
+    assert f(P, P, P, 2, P, None, None) == NULL
+    assert f(P, P, P + 2, 2, P, P, None) == ALIGN
 
 
 def test_frames_argument_checks(L):
