@@ -186,25 +186,56 @@ __device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) { return __fadd2_rn(a,
 __device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) { return __ffma2_rn(a, b, c); }
 
 // Eight consecutive elements, starting at element `elem`, of a per-sequence
-// vector stored as bf16 (F32 false) or fp32 (F32 true), as four fp32 pairs.
-// These vectors are shared by every row of a sequence: read-only path.
+// vector stored as bf16 (F32 false) or fp32 (F32 true).  These vectors are
+// shared by every row of a sequence: read-only path.  vec8_load only issues
+// the load(s) and keeps the raw words, so a loop can put every load of a step
+// in flight before the first conversion; vec8_unpack widens them to four fp32
+// pairs.
+template <bool F32>
+struct Vec8Raw;
+template <>
+struct Vec8Raw<false> {
+    uint4 u;
+};
+template <>
+struct Vec8Raw<true> {
+    float4 a, b;
+};
+
+template <bool F32>
+__device__ __forceinline__ Vec8Raw<F32> vec8_load(const void* base, int64_t elem)
+{
+    Vec8Raw<F32> r;
+    if constexpr (F32) {
+        const float4* f = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+        r.a = __ldg(f);
+        r.b = __ldg(f + 1);
+    } else {
+        r.u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem));
+    }
+    return r;
+}
+
+template <bool F32>
+__device__ __forceinline__ void vec8_unpack(const Vec8Raw<F32>& r, f32x2 (&v)[4])
+{
+    if constexpr (F32) {
+        v[0] = make_float2(r.a.x, r.a.y);
+        v[1] = make_float2(r.a.z, r.a.w);
+        v[2] = make_float2(r.b.x, r.b.y);
+        v[3] = make_float2(r.b.z, r.b.w);
+    } else {
+        v[0] = f2_from_bf16x2(r.u.x);
+        v[1] = f2_from_bf16x2(r.u.y);
+        v[2] = f2_from_bf16x2(r.u.z);
+        v[3] = f2_from_bf16x2(r.u.w);
+    }
+}
+
 template <bool F32>
 __device__ __forceinline__ void vec8_pairs(const void* base, int64_t elem, f32x2 (&v)[4])
 {
-    if (F32) {
-        const float4* f = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
-        const float4 a = __ldg(f), b = __ldg(f + 1);
-        v[0] = make_float2(a.x, a.y);
-        v[1] = make_float2(a.z, a.w);
-        v[2] = make_float2(b.x, b.y);
-        v[3] = make_float2(b.z, b.w);
-    } else {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem));
-        v[0] = f2_from_bf16x2(u.x);
-        v[1] = f2_from_bf16x2(u.y);
-        v[2] = f2_from_bf16x2(u.z);
-        v[3] = f2_from_bf16x2(u.w);
-    }
+    vec8_unpack<F32>(vec8_load<F32>(base, elem), v);
 }
 
 // fp32 pair -> bf16x2 word, round to nearest even.
@@ -242,10 +273,10 @@ __device__ __forceinline__ void team_barrier(int team)
 
 // Minimum resident CTAs per SM to ask of a row kernel holding VPT 16-byte
 // vectors per lane of each of INPUTS streamed inputs at once (about
-// 4 * INPUTS * VPT + 28 registers per thread).
-template <int VPT, int INPUTS = 1>
+// 4 * INPUTS * VPT + EXTRA registers per thread).
+template <int VPT, int INPUTS = 1, int EXTRA = 28>
 struct MinCtas {
-    static constexpr int regs = 4 * INPUTS * VPT + 28;
+    static constexpr int regs = 4 * INPUTS * VPT + EXTRA;
     static constexpr int raw = 65536 / (kCtaThreads * regs);
     static constexpr int value = raw < 1 ? 1 : (raw > 8 ? 8 : raw);
 };

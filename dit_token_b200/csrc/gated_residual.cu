@@ -38,14 +38,14 @@ gated_residual_kernel(const GatedParams p)
 
     for (int c0 = 0; c0 < nvec; c0 += kWarp * kUnroll) {
         uint4 xv[kUnroll], yv[kUnroll];
-        f32x2 gv[kUnroll][4];
+        Vec8Raw<F32> gv[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int j = c0 + u * kWarp + lane;
             if (j < nvec) {
                 xv[u] = ld_stream(xr + 8 * j);
                 yv[u] = ld_stream(yr + 8 * j);
-                vec8_pairs<F32>(p.gate, goff + 8 * j, gv[u]);
+                gv[u] = vec8_load<F32>(p.gate, goff + 8 * j);
             }
         }
 #pragma unroll
@@ -54,10 +54,12 @@ gated_residual_kernel(const GatedParams p)
             if (j < nvec) {
                 const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
                 const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
+                f32x2 g[4];
+                vec8_unpack<F32>(gv[u], g);
                 uint32_t o[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    o[e] = f2_to_bf16x2(f2_fma(gv[u][e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
+                    o[e] = f2_to_bf16x2(f2_fma(g[e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
                 st_stream(orow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
             }
         }

@@ -5,15 +5,14 @@
 // embedding; bullet 1: rotary rows are computed only where needed).
 //
 // Layout.  One warp per valid row.  A head of D = 8*LPH elements (D = 64,
-// 128 or 256) is held by a group of LPH lanes, 8 elements (one 16-byte vector)
-// per lane, so the per-head sum of squares is a log2(LPH)-step xor-shuffle
-// reduction.  A lane always sits at the same offset inside a head, so it
-// needs the cos/sin of only its own pairs (4 interleaved, 8 half-split): it
-// computes them once per row (angle reduced in fp64, then sincosf) and reuses
-// them for all num_q_heads + num_k_heads heads of that row -- cos/sin are
-// never re-read or recomputed per head.  Each step issues U head vectors per lane before any
-// arithmetic.  HBM traffic: q and k are each read once and written once, 4
-// bytes per element.
+// 128 or 256) is held by a group of LPH lanes, 8 elements per lane, so the
+// per-head sum of squares is a log2(LPH)-step xor-shuffle reduction.  A lane
+// always sits at the same place inside a head, so it needs the cos/sin of
+// only its own 4 pairs: it computes them once per row (angle reduced in fp64,
+// then sincosf) and reuses them for all num_q_heads + num_k_heads heads of
+// that row -- cos/sin are never re-read or recomputed per head.  Each step
+// issues U heads' loads per lane before any arithmetic.  HBM traffic: q and k
+// are each read once and written once, 4 bytes per element.
 #include "common.cuh"
 #include "launch.h"
 
@@ -35,25 +34,76 @@ __device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
     sincosf((float)red, &s, &c);
 }
 
-// Rotary layouts (template MODE): pair j of a head is (2j, 2j+1) when
-// interleaved -- all four of a lane's pairs are inside its own 8 elements --
-// or (j, j + D/2) when half-split -- a lane then holds one side of 8 pairs and
-// the lane LPH/2 away holds the other side, fetched with one xor shuffle per
-// element.  MODE none applies the RMSNorm and the weight only.
-//
-// Interleaved (the common case) folds the weight into the rotation: per lane
-// and per pair the four coefficients w0 cos, -w1 sin, w0 sin, w1 cos are formed
-// once per row (for q and for k), so a pair costs 2 multiplies and 2 FMAs plus
-// the RMS scale: (o0, o1) = r * (x0 w0 c - x1 w1 s, x0 w0 s + x1 w1 c).
+// Rotary layouts (template MODE).  In both rotating layouts a lane owns the
+// four pairs j = 4*li .. 4*li+3 of its head:
+//   interleaved  pair j = elements (2j, 2j+1): the lane's 16-byte vector
+//                 8*li .. 8*li+7 holds all four pairs;
+//   half-split   pair j = elements (j, j + D/2): the lane loads two 8-byte
+//                 vectors, elements 4*li .. 4*li+3 and D/2 + 4*li .. +3, so
+//                 both sides of each pair are its own and no lane exchange is
+//                 needed (a warp's 8-byte accesses still cover whole
+//                 128-byte lines).
+// Either way the weight is folded into the rotation: per lane and per pair the
+// four coefficients w0 cos, -w1 sin, w0 sin, w1 cos are formed once per row
+// (for q and for k), so a pair costs 2 multiplies and 2 FMAs plus the RMS
+// scale: (o0, o1) = r * (x0 w0 c - x1 w1 s, x0 w0 s + x1 w1 c), where w0, w1
+// are the weights of the pair's two elements.  MODE none applies the RMSNorm
+// and the weight only.
 
 struct PairCoef {
     float c00[4], c01[4], c10[4], c11[4];  // o0 = x0 c00 + x1 c01; o1 = x0 c10 + x1 c11
 };
 
-template <int D, int MODE, int NP>
-__device__ __forceinline__ void rms_rotate_heads(uint16_t* base, int H, int sub, float eps, const float (&w)[8],
-                                                 const PairCoef& pc, const float (&cs)[NP], const float (&sn)[NP],
-                                                 bool upper)
+// Element offset (from the head's start) of the lane's first / second access.
+template <int D, int MODE>
+__device__ __forceinline__ int lane_off(int li, int part)
+{
+    if (MODE == kRopeHalf)
+        return part * (D / 2) + 4 * li;
+    return 8 * li;
+}
+
+template <int D, int MODE>
+__device__ __forceinline__ uint4 load_head(const uint16_t* head, int li)
+{
+    if (MODE == kRopeHalf) {
+        const uint2 a = __ldcs(reinterpret_cast<const uint2*>(head + lane_off<D, MODE>(li, 0)));
+        const uint2 b = __ldcs(reinterpret_cast<const uint2*>(head + lane_off<D, MODE>(li, 1)));
+        return make_uint4(a.x, a.y, b.x, b.y);
+    }
+    return ld_stream(head + lane_off<D, MODE>(li, 0));
+}
+
+template <int D, int MODE>
+__device__ __forceinline__ void store_head(uint16_t* head, int li, uint4 v)
+{
+    if (MODE == kRopeHalf) {
+        __stcs(reinterpret_cast<uint2*>(head + lane_off<D, MODE>(li, 0)), make_uint2(v.x, v.y));
+        __stcs(reinterpret_cast<uint2*>(head + lane_off<D, MODE>(li, 1)), make_uint2(v.z, v.w));
+        return;
+    }
+    st_stream(head + lane_off<D, MODE>(li, 0), v);
+}
+
+// The lane's 8 elements in register order: interleaved (and none) = the
+// vector's own order; half-split = 4 elements of the first half, then the 4
+// matching elements of the second half.  Pair e of the lane is
+//   interleaved: registers (2e, 2e+1);  half-split: registers (e, 4+e).
+template <int MODE>
+__device__ __forceinline__ void pair_regs(int e, int& a, int& b)
+{
+    if (MODE == kRopeHalf) {
+        a = e;
+        b = 4 + e;
+    } else {
+        a = 2 * e;
+        b = 2 * e + 1;
+    }
+}
+
+template <int D, int MODE>
+__device__ __forceinline__ void rms_rotate_heads(uint16_t* row, int H, int sub, int li, float eps,
+                                                 const float (&w)[8], const PairCoef& pc)
 {
     constexpr int LPH = D / 8;
     constexpr int HPW = kWarp / LPH;
@@ -63,7 +113,7 @@ __device__ __forceinline__ void rms_rotate_heads(uint16_t* base, int H, int sub,
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int h = h0 + u * HPW + sub;
-            xv[u] = h < H ? ld_stream(base + (int64_t)h * D) : make_uint4(0u, 0u, 0u, 0u);
+            xv[u] = h < H ? load_head<D, MODE>(row + (int64_t)h * D, li) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -77,36 +127,23 @@ __device__ __forceinline__ void rms_rotate_heads(uint16_t* base, int H, int sub,
             }
             const float ss = group_sum<LPH>(ss2.x + ss2.y);  // every lane of the warp takes part
             const float r = rsqrtf(ss * inv_d + eps);
-            float o[8];
-            if (MODE == kRopeInterleaved) {
+            float x[8], o[8];
+            unpack8(xv[u], x);
+            if (MODE == kRopeNone) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = bf16_lo(wd[e]), x1 = bf16_hi(wd[e]);
-                    o[2 * e] = r * fmaf(x1, pc.c01[e], x0 * pc.c00[e]);
-                    o[2 * e + 1] = r * fmaf(x1, pc.c11[e], x0 * pc.c10[e]);
-                }
+                for (int e = 0; e < 8; ++e)
+                    o[e] = x[e] * (r * w[e]);
             } else {
-                float y[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    y[2 * e] = bf16_lo(wd[e]) * (r * w[2 * e]);
-                    y[2 * e + 1] = bf16_hi(wd[e]) * (r * w[2 * e + 1]);
-                }
-                if (MODE == kRopeHalf) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float partner = __shfl_xor_sync(0xffffffffu, y[e], LPH / 2);  // all lanes take part
-                        o[e] = upper ? partner * sn[e % NP] + y[e] * cs[e % NP]
-                                     : y[e] * cs[e % NP] - partner * sn[e % NP];
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o[e] = y[e];
+                    int a, b;
+                    pair_regs<MODE>(e, a, b);
+                    o[a] = r * fmaf(x[b], pc.c01[e], x[a] * pc.c00[e]);
+                    o[b] = r * fmaf(x[b], pc.c11[e], x[a] * pc.c10[e]);
                 }
             }
             if (h < H)
-                st_stream(base + (int64_t)h * D, pack8(o));
+                store_head<D, MODE>(row + (int64_t)h * D, li, pack8(o));
         }
     }
 }
@@ -116,7 +153,7 @@ __global__ void __launch_bounds__(kCtaThreads)
 qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
 {
     constexpr int LPH = D / 8;          // lanes per head
-    constexpr int NP = MODE == kRopeHalf ? 8 : (MODE == kRopeInterleaved ? 4 : 1);  // pairs per lane
+    constexpr int NP = MODE == kRopeNone ? 1 : 4;  // pairs per lane
     const int lane = threadIdx.x & (kWarp - 1);
     const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     RowSlot s;
@@ -124,8 +161,7 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
                        p.pk.num_rows_padded, lane, s))
         return;
     const int sub = lane / LPH;  // which head of the step
-    const int li = lane % LPH;   // position inside the head: elements 8*li .. 8*li+7
-    const bool upper = MODE == kRopeHalf && li >= LPH / 2;  // holds the j + D/2 side
+    const int li = lane % LPH;   // position inside the head: pairs 4*li .. 4*li+3
 
     float cs[NP], sn[NP];
 #pragma unroll
@@ -156,35 +192,47 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         }
 #pragma unroll
         for (int e = 0; e < NP; ++e) {
-            const int j = MODE == kRopeHalf ? 8 * (li % (LPH / 2)) + e : 4 * li + e;
+            const int j = 4 * li + e;
             const int ax = p.axis[j];
             const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
             const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
             pair_cos_sin(ang, cs[e], sn[e]);
         }
     }
+    // the weights of the lane's 8 elements, in register order
     float wq[8], wk[8];
-    unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
-    unpack8(ld_shared_vec(p.k_weight + 8 * li), wk);
+    if (MODE == kRopeHalf) {
+        const uint2 q0 = __ldg(reinterpret_cast<const uint2*>(p.q_weight + lane_off<D, MODE>(li, 0)));
+        const uint2 q1 = __ldg(reinterpret_cast<const uint2*>(p.q_weight + lane_off<D, MODE>(li, 1)));
+        const uint2 k0 = __ldg(reinterpret_cast<const uint2*>(p.k_weight + lane_off<D, MODE>(li, 0)));
+        const uint2 k1 = __ldg(reinterpret_cast<const uint2*>(p.k_weight + lane_off<D, MODE>(li, 1)));
+        unpack8(make_uint4(q0.x, q0.y, q1.x, q1.y), wq);
+        unpack8(make_uint4(k0.x, k0.y, k1.x, k1.y), wk);
+    } else {
+        unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
+        unpack8(ld_shared_vec(p.k_weight + 8 * li), wk);
+    }
     PairCoef pq{}, pk{};
-    if (MODE == kRopeInterleaved) {
+    if (MODE != kRopeNone) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+            int a, b;
+            pair_regs<MODE>(e, a, b);
             const float c = cs[e % NP], sv = sn[e % NP];
-            pq.c00[e] = wq[2 * e] * c;
-            pq.c01[e] = -wq[2 * e + 1] * sv;
-            pq.c10[e] = wq[2 * e] * sv;
-            pq.c11[e] = wq[2 * e + 1] * c;
-            pk.c00[e] = wk[2 * e] * c;
-            pk.c01[e] = -wk[2 * e + 1] * sv;
-            pk.c10[e] = wk[2 * e] * sv;
-            pk.c11[e] = wk[2 * e + 1] * c;
+            pq.c00[e] = wq[a] * c;
+            pq.c01[e] = -wq[b] * sv;
+            pq.c10[e] = wq[a] * sv;
+            pq.c11[e] = wq[b] * c;
+            pk.c00[e] = wk[a] * c;
+            pk.c01[e] = -wk[b] * sv;
+            pk.c10[e] = wk[a] * sv;
+            pk.c11[e] = wk[b] * c;
         }
     }
-    uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride + 8 * li;
-    uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride + 8 * li;
-    rms_rotate_heads<D, MODE, NP>(qrow, p.num_q_heads, sub, p.eps, wq, pq, cs, sn, upper);
-    rms_rotate_heads<D, MODE, NP>(krow, p.num_k_heads, sub, p.eps, wk, pk, cs, sn, upper);
+    uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride;
+    uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride;
+    rms_rotate_heads<D, MODE>(qrow, p.num_q_heads, sub, li, p.eps, wq, pq);
+    rms_rotate_heads<D, MODE>(krow, p.num_k_heads, sub, li, p.eps, wk, pk);
 }
 
 template <int D>
