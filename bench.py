@@ -71,12 +71,22 @@ def algorithmic_bytes(w: W.Workload) -> dict:
             "gated_residual": 6 * w.hidden * n, "swiglu": 6 * w.inner * n}
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source with comments removed and whitespace collapsed: the digest
+    follows the code, not its commentary."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_digest(op: str) -> str:
-    path = os.path.join(ROOT, "dit_token_b200", "csrc", f"{op}.cu")
+    """Digest of the code of an op's kernel file, the shared device header and
+    the launch header (comments and layout ignored)."""
+    csrc = os.path.join(ROOT, "dit_token_b200", "csrc")
     h = hashlib.sha256()
-    for p in (path, os.path.join(ROOT, "dit_token_b200", "csrc", "common.cuh")):
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for name in (f"{op}.cu", "common.cuh", "launch.h"):
+        with open(os.path.join(csrc, name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -29,7 +29,12 @@
 // cp.async 370-450 us; persistent 4-warp CTAs with 3 rows prefetched in
 // registers 352 us; the row streamed twice (second read from L2) 339 us;
 // one warp per row with the next row prefetched into shared memory by
-// cp.async (modulation then from global) 316 us; this kernel 251-264 us.
+// cp.async (modulation then from global) 316 us; one warp per row fed by 1-D
+// bulk copies (TMA) into a 2-slot shared-memory ring per warp with mbarrier
+// completion, 8 warps and 205 KB of shared memory per SM, 523 us (ncu: 26 %
+// of DRAM peak, SM activity very uneven -- active cycles min / mean / max
+// 2k / 132k / 203k of 210k -- with the copy engine's pipe nearly idle); this
+// kernel 251-264 us.
 #include "common.cuh"
 #include "launch.h"
 
