@@ -34,7 +34,9 @@
 // completion, 8 warps and 205 KB of shared memory per SM, 523 us (ncu: 26 %
 // of DRAM peak, SM activity very uneven -- active cycles min / mean / max
 // 2k / 132k / 203k of 210k -- with the copy engine's pipe nearly idle); this
-// kernel 251-264 us.
+// kernel with each register vector refilled with the next row's during the
+// output pass 248 us against 244 us without (both with a clean L2); this
+// kernel 244-264 us.
 #include "common.cuh"
 #include "launch.h"
 
