@@ -730,7 +730,7 @@ def main(argv=None):
     ap.add_argument("--scale", type=float, default=1.0,
                     help="scale every sequence's valid length (a smaller batch of the same shapes, "
                          "e.g. for profiling); the JSON names the scaled workload")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true",
