@@ -42,6 +42,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_qk_rmsnorm_rope_ex.argtypes = [
             u16p, i64, u16p, i64, u16p, u16p, i32p, i32p, i32, i64, i32, i32, i32,
             i32p, i32, i32, i32, f64, f64, i32, u16p, u16p, f64p, f64p, i64p, i64]
+        L.oracle_qk_rmsnorm_rope_shard.argtypes = [
+            u16p, i64, u16p, i64, u16p, u16p, i32p, i32p, i32, i64, i32, i32, i32,
+            i32p, i32, i32, i32, f64, f64, i32, i32p, u16p, u16p, f64p, f64p, i64p, i64]
         L.oracle_adaln_modulate.argtypes = [
             u16p, i64, u16p, u16p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
         L.oracle_gated_residual.argtypes = [
@@ -58,12 +61,12 @@ def lib() -> ctypes.CDLL:
             u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i32p, i32, i64, i32, f64,
             u16p, i64, u16p, i64, f64p, i64p, i64]
         L.oracle_adaln_modulate_av.argtypes = [
-            u16p, i64, vp, vp, i64, i32, i32p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
+            u16p, i64, vp, vp, i64, i32, i32p, i32p, i64, i32p, i32p, i32, i64, i32, f64, u16p, i64, f64p, i64p, i64]
         L.oracle_gated_residual_av.argtypes = [
-            u16p, i64, u16p, i64, vp, i64, i32, i32p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p,
+            u16p, i64, u16p, i64, vp, i64, i32, i32p, i32p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p,
             i64]
         L.oracle_gated_residual_adaln_av.argtypes = [
-            u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i64, i64, i32p, i32p, i32, i64, i32, f64,
+            u16p, i64, u16p, i64, vp, i64, vp, vp, i64, i32, i32p, i32p, i64, i64, i32p, i32p, i32, i64, i32, f64,
             u16p, i64, u16p, i64, f64p, i64p, i64]
         L.oracle_swiglu.argtypes = [
             u16p, i64, u16p, i64, i32p, i32p, i32, i64, i32, u16p, i64, f64p, i64p, i64]
@@ -74,6 +77,7 @@ def lib() -> ctypes.CDLL:
                      "oracle_gated_residual", "oracle_gated_residual_adaln", "oracle_swiglu",
                      "oracle_adaln_modulate_ex", "oracle_gated_residual_ex", "oracle_gated_residual_adaln_ex",
                      "oracle_adaln_modulate_av", "oracle_gated_residual_av", "oracle_gated_residual_adaln_av",
+                     "oracle_qk_rmsnorm_rope_shard",
                      "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -163,11 +167,13 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
                     sections=(0, 0, 0), rope_theta=10000.0, eps=1e-6,
                     q_row_stride=None, k_row_stride=None, rows=None,
                     q_out_init=None, k_out_init=None, want_f64=False, q_out=None, k_out=None,
-                    rope_mode="interleaved"):
+                    rope_mode="interleaved", pos_offset=None):
     """Per-head Q/K RMSNorm fused with 1D / 3D rotary embedding.
 
     rope_mode: "interleaved" (pairs 2j, 2j+1), "half" (pairs j, j + D/2) or
-    "none" (RMSNorm only).
+    "none" (RMSNorm only).  pos_offset: int32 [num_seqs] or None -- the rows
+    of sequence b are rows pos_offset[b], ... of the whole sequence (one
+    rank's slice).
 
     q, k: uint16 arrays whose first axis is the padded row; row strides
     default to the product of the remaining axes.  Returns (q_out, k_out) or,
@@ -189,12 +195,14 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
     r, nr = _rows(rows)
     L = lib()
     mode = {"interleaved": 0, "half": 1, "none": 2}[rope_mode]
-    rc = L.oracle_qk_rmsnorm_rope_ex(
+    po = _int32(pos_offset)
+    rc = L.oracle_qk_rmsnorm_rope_shard(
         _ptr(q, ctypes.c_uint16), qs, _ptr(k, ctypes.c_uint16), ks,
         _ptr(wq, ctypes.c_uint16), _ptr(wk, ctypes.c_uint16),
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows,
         num_q_heads, num_k_heads, head_dim,
         _ptr(grid, ctypes.c_int32), *[int(s) for s in sections], float(rope_theta), float(eps), mode,
+        _ptr(po, ctypes.c_int32),
         _ptr(q_out, ctypes.c_uint16), _ptr(k_out, ctypes.c_uint16),
         _ptr(q64, ctypes.c_double), _ptr(k64, ctypes.c_double),
         _ptr(r, ctypes.c_int64), nr)
@@ -204,20 +212,22 @@ def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,
     return q_out, k_out
 
 
-def _grid(rope_grid):
-    return None if rope_grid is None else np.ascontiguousarray(np.asarray(rope_grid, dtype=np.int32))
+def _int32(a):
+    """A contiguous int32 copy of an optional integer array (grids, offsets)."""
+    return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.int32))
 
 
 def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
                    mod_seq_stride=None, x_row_stride=None, rows=None, out_init=None,
-                   want_f64=False, out=None, rope_grid=None, audio_offset=0):
+                   want_f64=False, out=None, rope_grid=None, audio_offset=0, pos_offset=None):
     """out = LayerNorm(x) * (1 + scale_b) + shift_b on valid rows.
 
     shift, scale: uint16 (bf16 bits) or float32 arrays [num_seqs, ...] read
     with mod_seq_stride elements between sequences (default: hidden).
     Per-stream vectors: with rope_grid [num_seqs][3] given, the audio rows of
     sequence b (local index >= T*H*W) read their vectors audio_offset
-    elements after the video rows' ones."""
+    elements after the video rows' ones; pos_offset [num_seqs] (or None) is
+    where each sequence's rows start in the whole sequence."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
     B = cs.size - 1
     x, xs = _flat_view(x, x_row_stride, None)
@@ -231,9 +241,10 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
         raise TypeError("shift and scale must have the same dtype")
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    grid = _grid(rope_grid)
+    grid = _int32(rope_grid)
     rc = lib().oracle_adaln_modulate_av(
-        _ptr(x, ctypes.c_uint16), xs, _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32), audio_offset,
+        _ptr(x, ctypes.c_uint16), xs, _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32),
+        _ptr(_int32(pos_offset), ctypes.c_int32), audio_offset,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "adaln_modulate")
@@ -242,7 +253,7 @@ def adaln_modulate(x, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, ep
 
 def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_seq_stride=None,
                    x_row_stride=None, y_row_stride=None, rows=None, out_init=None,
-                   want_f64=False, out=None, rope_grid=None, audio_offset=0):
+                   want_f64=False, out=None, rope_grid=None, audio_offset=0, pos_offset=None):
     """out = x + gate_b * y on valid rows (per-stream gates as in
     adaln_modulate)."""
     cs, cp = _seqlens(cu_seqlens, cu_seqlens_padded)
@@ -256,10 +267,11 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
     g, gf = _mod(gate)
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     r, nr = _rows(rows)
-    grid = _grid(rope_grid)
+    grid = _int32(rope_grid)
     rc = lib().oracle_gated_residual_av(
         _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss, gf,
-        _ptr(grid, ctypes.c_int32), audio_offset, _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
+        _ptr(grid, ctypes.c_int32), _ptr(_int32(pos_offset), ctypes.c_int32), audio_offset,
+        _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden,
         _ptr(out, ctypes.c_uint16), xs, _ptr(o64, ctypes.c_double), _ptr(r, ctypes.c_int64), nr)
     _check(rc, "gated_residual")
     return (out, o64) if want_f64 else out
@@ -268,7 +280,8 @@ def gated_residual(x, y, gate, cu_seqlens, cu_seqlens_padded, *, hidden, gate_se
 def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded, *, hidden, eps=1e-6,
                         gate_seq_stride=None, mod_seq_stride=None, x_row_stride=None, y_row_stride=None,
                         rows=None, res_init=None, norm_init=None, want_f64=False, res_out=None,
-                        norm_out=None, rope_grid=None, gate_audio_offset=0, mod_audio_offset=0):
+                        norm_out=None, rope_grid=None, gate_audio_offset=0, mod_audio_offset=0,
+                        pos_offset=None):
     """res = x + gate_b * y (bf16), norm = LN(res) * (1 + scale_b) + shift_b on
     valid rows (per-stream vectors as in adaln_modulate, with one audio
     offset for the gate and one for shift/scale).  Returns (res, norm) or,
@@ -291,10 +304,11 @@ def gated_residual_adaln(x, y, gate, shift, scale, cu_seqlens, cu_seqlens_padded
     gss = hidden if gate_seq_stride is None else gate_seq_stride
     mss = hidden if mod_seq_stride is None else mod_seq_stride
     r, nr = _rows(rows)
-    grid = _grid(rope_grid)
+    grid = _int32(rope_grid)
     rc = lib().oracle_gated_residual_adaln_av(
         _ptr(x, ctypes.c_uint16), xs, _ptr(y, ctypes.c_uint16), ys, _vptr(g), gss,
-        _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32), gate_audio_offset, mod_audio_offset,
+        _vptr(sh), _vptr(sc), mss, f1, _ptr(grid, ctypes.c_int32), _ptr(_int32(pos_offset), ctypes.c_int32),
+        gate_audio_offset, mod_audio_offset,
         _ptr(cs, ctypes.c_int32), _ptr(cp, ctypes.c_int32), B, nrows, hidden, float(eps),
         _ptr(res_out, ctypes.c_uint16), xs, _ptr(norm_out, ctypes.c_uint16), xs, _ptr(n64, ctypes.c_double),
         _ptr(r, ctypes.c_int64), nr)

@@ -83,14 +83,17 @@ static double ldm(const void* base, int64_t idx, int f32)
  * One vector set per sequence: b * seq_stride.  With per-stream vectors
  * (rope_grid != NULL) the joint audio-video sequence holds its T*H*W video
  * rows first and its audio rows after them; video rows use the set at
- * b * seq_stride, audio rows the set audio_offset elements further on. */
+ * b * seq_stride, audio rows the set audio_offset elements further on.  A row's
+ * index in its whole sequence is its local index plus the sequence's position
+ * offset (pos_offset NULL: 0). */
 static int64_t vec_offset(int32_t b, int64_t r, int64_t seq_stride, const int32_t* rope_grid,
-                          int64_t audio_offset)
+                          const int32_t* pos_offset, int64_t audio_offset)
 {
     int64_t off = (int64_t)b * seq_stride;
     if (rope_grid) {
         int64_t thw = (int64_t)rope_grid[3 * b] * rope_grid[3 * b + 1] * rope_grid[3 * b + 2];
-        if (r >= thw)
+        int64_t g = r + (pos_offset ? pos_offset[b] : 0); /* index in the whole sequence */
+        if (g >= thw)
             off += audio_offset;
     }
     return off;
@@ -235,6 +238,24 @@ int oracle_qk_rmsnorm_rope_ex(
     uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
     const int64_t* rows, int64_t num_rows)
 {
+    return oracle_qk_rmsnorm_rope_shard(q, q_row_stride, k, k_row_stride, q_weight, k_weight, cu_seqlens,
+                                        cu_seqlens_padded, num_seqs, num_rows_padded, num_q_heads, num_k_heads,
+                                        head_dim, rope_grid, sec_t, sec_h, sec_w, rope_theta, eps, rope_mode, NULL,
+                                        q_out, k_out, q_out_f64, k_out_f64, rows, num_rows);
+}
+
+int oracle_qk_rmsnorm_rope_shard(
+    const uint16_t* q, int64_t q_row_stride,
+    const uint16_t* k, int64_t k_row_stride,
+    const uint16_t* q_weight, const uint16_t* k_weight,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded,
+    int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+    const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+    double rope_theta, double eps, int32_t rope_mode, const int32_t* pos_offset,
+    uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
+    const int64_t* rows, int64_t num_rows)
+{
     if (!q || !k || !q_weight || !k_weight || !q_out || !k_out)
         return -1;
     if (rope_mode != ORACLE_ROPE_INTERLEAVED && rope_mode != ORACLE_ROPE_HALF && rope_mode != ORACLE_ROPE_NONE)
@@ -266,21 +287,25 @@ int oracle_qk_rmsnorm_rope_ex(
                 continue;
             if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
                 continue;
-            /* Positions: a row inside the sequence's T x H x W video grid
-             * (t-major, then h, then w) takes 3D positions; every other row
-             * takes the 1D position counted from the end of the grid. */
+            /* Positions: the row's index in its whole sequence is g = r plus
+             * the sequence's position offset (non-zero when this buffer holds
+             * one rank's slice of a longer sequence).  A row inside the
+             * sequence's T x H x W video grid (t-major, then h, then w) takes
+             * 3D positions; every other row takes the 1D position counted
+             * from the end of the grid. */
+            const int64_t g = r + (pos_offset ? pos_offset[b] : 0);
             int is3d = 0;
-            int64_t pos3[3] = {0, 0, 0}, pos1 = r;
+            int64_t pos3[3] = {0, 0, 0}, pos1 = g;
             if (rope_grid) {
                 int64_t T = rope_grid[3 * b], H = rope_grid[3 * b + 1], W = rope_grid[3 * b + 2];
                 int64_t thw = T * H * W;
-                if (r < thw) {
+                if (g < thw) {
                     is3d = 1;
-                    pos3[0] = r / (H * W);
-                    pos3[1] = (r / W) % H;
-                    pos3[2] = r % W;
+                    pos3[0] = g / (H * W);
+                    pos3[1] = (g / W) % H;
+                    pos3[2] = g % W;
                 } else {
-                    pos1 = r - thw;
+                    pos1 = g - thw;
                 }
             }
             for (int32_t h = 0; h < num_q_heads; ++h) {
@@ -321,7 +346,7 @@ int oracle_adaln_modulate_ex(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows)
 {
-    return oracle_adaln_modulate_av(x, x_row_stride, shift, scale, mod_seq_stride, mod_f32, NULL, 0, cu_seqlens,
+    return oracle_adaln_modulate_av(x, x_row_stride, shift, scale, mod_seq_stride, mod_f32, NULL, NULL, 0, cu_seqlens,
                                     cu_seqlens_padded, num_seqs, num_rows_padded, hidden, eps, out,
                                     out_row_stride, out_f64, rows, num_rows);
 }
@@ -329,7 +354,7 @@ int oracle_adaln_modulate_ex(
 int oracle_adaln_modulate_av(
     const uint16_t* x, int64_t x_row_stride,
     const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
-    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
@@ -352,7 +377,7 @@ int oracle_adaln_modulate_av(
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
         const uint16_t* xr = x + row * x_row_stride;
-        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, audio_offset);
+        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, pos_offset, audio_offset);
         /* LayerNorm without affine: mean, then the biased variance about it. */
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
@@ -398,7 +423,7 @@ int oracle_gated_residual_ex(
     uint16_t* out, int64_t out_row_stride, double* out_f64,
     const int64_t* rows, int64_t num_rows)
 {
-    return oracle_gated_residual_av(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, gate_f32, NULL, 0,
+    return oracle_gated_residual_av(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, gate_f32, NULL, NULL, 0,
                                     cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, hidden, out,
                                     out_row_stride, out_f64, rows, num_rows);
 }
@@ -407,7 +432,7 @@ int oracle_gated_residual_av(
     const uint16_t* x, int64_t x_row_stride,
     const uint16_t* y, int64_t y_row_stride,
     const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
-    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
@@ -429,7 +454,7 @@ int oracle_gated_residual_av(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, audio_offset);
+        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, pos_offset, audio_offset);
         for (int32_t c = 0; c < hidden; ++c) {
             double v = ld(&x[row * x_row_stride + c]) + ldm(gate, gb + c, gate_f32) * ld(&y[row * y_row_stride + c]);
             put(out, out_f64, row * out_row_stride + c, v);
@@ -475,7 +500,7 @@ int oracle_gated_residual_adaln_ex(
     const int64_t* rows, int64_t num_rows)
 {
     return oracle_gated_residual_adaln_av(x, x_row_stride, y, y_row_stride, gate, gate_seq_stride, shift, scale,
-                                          mod_seq_stride, mod_f32, NULL, 0, 0, cu_seqlens, cu_seqlens_padded,
+                                          mod_seq_stride, mod_f32, NULL, NULL, 0, 0, cu_seqlens, cu_seqlens_padded,
                                           num_seqs, num_rows_padded, hidden, eps, res_out, res_row_stride,
                                           norm_out, norm_row_stride, norm_out_f64, rows, num_rows);
 }
@@ -485,7 +510,7 @@ int oracle_gated_residual_adaln_av(
     const uint16_t* y, int64_t y_row_stride,
     const void* gate, int64_t gate_seq_stride,
     const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
-    const int32_t* rope_grid, int64_t gate_audio_offset, int64_t mod_audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t gate_audio_offset, int64_t mod_audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
     uint16_t* res_out, int64_t res_row_stride,
@@ -509,7 +534,7 @@ int oracle_gated_residual_adaln_av(
             continue;
         if (!locate_row(cu_seqlens, cu_seqlens_padded, num_seqs, row, &b, &r))
             continue;
-        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, gate_audio_offset);
+        const int64_t gb = vec_offset(b, r, gate_seq_stride, rope_grid, pos_offset, gate_audio_offset);
         uint16_t* rr = res_out + row * res_row_stride;
         /* step 1: residual update, stored as bf16 */
         for (int32_t c = 0; c < hidden; ++c) {
@@ -517,7 +542,7 @@ int oracle_gated_residual_adaln_av(
             rr[c] = oracle_f64_to_bf16(v);
         }
         /* step 2: adaLN of the stored residual */
-        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, mod_audio_offset);
+        const int64_t mb = vec_offset(b, r, mod_seq_stride, rope_grid, pos_offset, mod_audio_offset);
         double mean = 0.0;
         for (int32_t c = 0; c < hidden; ++c)
             mean += ld(&rr[c]);

@@ -88,6 +88,24 @@ int oracle_qk_rmsnorm_rope_ex(
     uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
     const int64_t* rows, int64_t num_rows);
 
+/* oracle_qk_rmsnorm_rope_ex on one rank's slice of longer sequences: the
+ * rows of sequence b are the rows pos_offset[b], pos_offset[b] + 1, ... of
+ * the whole sequence, and take that sequence's positions (3D inside its grid,
+ * 1D after it).  The pages restrict each rank's rotary work to its own rows
+ * ("Why Real-Time MiniMax H3 Serving Requires More Than a Faster DiT", "Key
+ * takeaways", bullet 1).  pos_offset NULL is the _ex function. */
+int oracle_qk_rmsnorm_rope_shard(
+    const uint16_t* q, int64_t q_row_stride,
+    const uint16_t* k, int64_t k_row_stride,
+    const uint16_t* q_weight, const uint16_t* k_weight,
+    const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+    int32_t num_seqs, int64_t num_rows_padded,
+    int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+    const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+    double rope_theta, double eps, int32_t rope_mode, const int32_t* pos_offset,
+    uint16_t* q_out, uint16_t* k_out, double* q_out_f64, double* k_out_f64,
+    const int64_t* rows, int64_t num_rows);
+
 /* Adaptive LayerNorm modulation: out = LN(x) * (1 + scale_b) + shift_b.
  * shift/scale: bf16[num_seqs][hidden] with a per-sequence stride of
  * mod_seq_stride elements. */
@@ -159,12 +177,14 @@ int oracle_gated_residual_adaln_ex(
  * bullet 1; they do not say whether the two streams share modulation
  * vectors).  Sequence b holds rope_grid[b] = (T, H, W): its first T*H*W valid
  * rows are video and use the vectors at b * stride; the remaining valid rows
- * are audio and use the vectors audio_offset elements further on.  With
- * rope_grid NULL every row uses b * stride (the _ex functions). */
+ * are audio and use the vectors audio_offset elements further on.  A row's
+ * index in its whole sequence is its local index plus pos_offset[b]
+ * (pos_offset NULL: 0), as in oracle_qk_rmsnorm_rope_shard.  With rope_grid
+ * NULL every row uses b * stride (the _ex functions). */
 int oracle_adaln_modulate_av(
     const uint16_t* x, int64_t x_row_stride,
     const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
-    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
@@ -173,7 +193,7 @@ int oracle_gated_residual_av(
     const uint16_t* x, int64_t x_row_stride,
     const uint16_t* y, int64_t y_row_stride,
     const void* gate, int64_t gate_seq_stride, int32_t gate_f32,
-    const int32_t* rope_grid, int64_t audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden,
     uint16_t* out, int64_t out_row_stride, double* out_f64,
@@ -183,7 +203,7 @@ int oracle_gated_residual_adaln_av(
     const uint16_t* y, int64_t y_row_stride,
     const void* gate, int64_t gate_seq_stride,
     const void* shift, const void* scale, int64_t mod_seq_stride, int32_t mod_f32,
-    const int32_t* rope_grid, int64_t gate_audio_offset, int64_t mod_audio_offset,
+    const int32_t* rope_grid, const int32_t* pos_offset, int64_t gate_audio_offset, int64_t mod_audio_offset,
     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
     int32_t num_seqs, int64_t num_rows_padded, int32_t hidden, double eps,
     uint16_t* res_out, int64_t res_row_stride,

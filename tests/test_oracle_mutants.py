@@ -18,7 +18,8 @@ SRC = os.path.join(ROOT, "oracle", "oracle.c")
 PINS = ["tests/test_oracle_bf16.py", "tests/test_oracle_qk.py", "tests/test_oracle_adaln.py",
         "tests/test_oracle_residual_swiglu.py", "tests/test_oracle_packing.py", "tests/test_oracle_fused.py",
         "tests/test_oracle_frames.py", "tests/test_oracle_rope_modes.py",
-        "tests/test_oracle_modulation_f32.py", "tests/test_oracle_av_modulation.py"]
+        "tests/test_oracle_modulation_f32.py", "tests/test_oracle_av_modulation.py",
+        "tests/test_oracle_shard.py"]
 
 # (name, original text, planted mistake)
 MUTANTS = [
@@ -33,8 +34,8 @@ MUTANTS = [
     ("rms_mean_not_divided", "ms /= (double)D;", ""),
     ("rms_weight_dropped", "y[i] = ld(&x[i]) * inv_rms * ld(&w[i]);", "y[i] = ld(&x[i]) * inv_rms;"),
     ("rope_3d_freq_whole_head", "(double)jl / (double)sec[s]", "(double)jl / (double)head_dim"),
-    ("rope_3d_h_index", "pos3[1] = (r / W) % H;", "pos3[1] = (r / H) % W;"),
-    ("rope_tail_position", "pos1 = r - thw;", "pos1 = r;"),
+    ("rope_3d_h_index", "pos3[1] = (g / W) % H;", "pos3[1] = (g / H) % W;"),
+    ("rope_tail_position", "pos1 = g - thw;", "pos1 = g;"),
     ("rope_k_uses_q_weight", "rmsnorm_rope_head(k + off, k_weight,", "rmsnorm_rope_head(k + off, q_weight,"),
     ("adaln_scale_without_one", "xhat * (1.0 + ldm(scale, mb + c, mod_f32))", "xhat * ldm(scale, mb + c, mod_f32)"),
     ("adaln_unbiased_variance", "var /= (double)hidden;", "var /= (double)(hidden - 1);"),
@@ -45,8 +46,12 @@ MUTANTS = [
     ("fused_gate_dropped", "ldm(gate, gb + c, mod_f32) * ld(&y[row * y_row_stride + c])",
      "ld(&y[row * y_row_stride + c])"),
     ("vectors_not_per_sequence", "int64_t off = (int64_t)b * seq_stride;", "int64_t off = 0;"),
-    ("audio_split_off_by_one", "if (r >= thw)\n            off += audio_offset;", "if (r > thw)\n            off += audio_offset;"),
+    ("audio_split_off_by_one", "if (g >= thw)\n            off += audio_offset;", "if (g > thw)\n            off += audio_offset;"),
     ("audio_vectors_ignored", "off += audio_offset;", "off += 0;"),
+    ("rope_position_offset_ignored", "const int64_t g = r + (pos_offset ? pos_offset[b] : 0);",
+     "const int64_t g = r;"),
+    ("stream_split_offset_ignored", "int64_t g = r + (pos_offset ? pos_offset[b] : 0); /* index in the whole sequence */",
+     "int64_t g = r;"),
     ("silu_sign", "exp(-av)", "exp(av)"),
     ("swiglu_operands_transposed", "double silu = av / (1.0 + exp(-av));\n            put(out, out_f64, row * out_row_stride + c, silu * bv);",
      "double silu = bv / (1.0 + exp(-bv));\n            put(out, out_f64, row * out_row_stride + c, silu * av);"),
