@@ -57,6 +57,8 @@ _SIGNATURES = {
                             _VP, _I32, _I32, _I32, _F32, _F32, _VP],
     "dit_qk_rmsnorm_rope_ex": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
                                _VP, _I32, _I32, _I32, _F32, _F32, _I32, _VP],
+    "dit_qk_rmsnorm_rope_shard": [_VP, _I64, _VP, _I64, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
+                                  _VP, _I32, _I32, _I32, _F32, _F32, _I32, _VP, _VP],
     "dit_adaln_modulate": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _VP],
     "dit_adaln_modulate_ex": [_VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _VP, _I32, _I64, _I32, _F32, _I32,
                               _VP],
@@ -69,7 +71,7 @@ _SIGNATURES = {
     "dit_gated_residual_adaln_ex": [_VP, _I64, _VP, _I64, _VP, _I64, _VP, _VP, _I64, _VP, _I64, _VP, _I64,
                                     _VP, _VP, _I32, _I64, _I32, _F32, _I32, _VP],
     "dit_validate_seqlens": [_VP, _VP, _I32, _I64, _VP, _VP],
-    "dit_av_stream_seqlens": [_VP, _VP, _VP, _I32, _VP, _VP, _VP],
+    "dit_av_stream_seqlens": [_VP, _VP, _VP, _VP, _I32, _VP, _VP, _VP],
     "dit_frames_to_u8": [_VP, _I64, _I64, _I64, _I64, _I64, _I32, _VP, _VP],
     "dit_status_string": [_I32],
     "dit_last_cuda_error": [],
@@ -168,7 +170,8 @@ def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor
                         num_q_heads: int, num_k_heads: int, head_dim: int,
                         rope_grid: Optional[torch.Tensor] = None,
                         sections: Sequence[int] = (0, 0, 0), rope_theta: float = 10000.0,
-                        eps: float = 1e-6, rope_mode: str = "interleaved", stream=None) -> None:
+                        eps: float = 1e-6, rope_mode: str = "interleaved",
+                        pos_offset: Optional[torch.Tensor] = None, stream=None) -> None:
     """In place: q, k <- RoPE(RMSNorm_head(q) * q_weight), RoPE(RMSNorm_head(k) * k_weight).
 
     q: [rows, num_q_heads * head_dim] (or [rows, heads, head_dim]) bf16, any
@@ -176,7 +179,9 @@ def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor
     (every row 1D); sections: t/h/w widths of head_dim on 3D rows.
     rope_mode: "interleaved" (pairs 2j, 2j+1; the C entry dit_qk_rmsnorm_rope),
     "half" (pairs j, j + D/2) or "none" (RMSNorm only) -- the latter two, and
-    head_dim 256, go through dit_qk_rmsnorm_rope_ex."""
+    head_dim 256, go through dit_qk_rmsnorm_rope_ex.  pos_offset: int32
+    [num_seqs] or None -- this buffer holds a slice of longer sequences whose
+    rows start at row pos_offset[b] of sequence b (dit_qk_rmsnorm_rope_shard)."""
     qp, qs = _rows(q, "q")
     kp, ks = _rows(k, "k")
     if k.size(0) != q.size(0):
@@ -192,10 +197,19 @@ def dit_qk_rmsnorm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor
     args = (qp, qs, kp, ks, _vec(q_weight, "q_weight"), _vec(k_weight, "k_weight"), cs, cp, B, q.size(0),
             num_q_heads, num_k_heads, head_dim, gp or None, st, sh, sw, float(rope_theta), float(eps))
     mode = {"interleaved": 0, "half": 1, "none": 2}[rope_mode]
-    if mode == 0 and head_dim in (64, 128):
+    if pos_offset is not None:
+        _call("dit_qk_rmsnorm_rope_shard", *args, mode, _offsets(pos_offset, B), _stream(stream))
+    elif mode == 0 and head_dim in (64, 128):
         _call("dit_qk_rmsnorm_rope", *args, _stream(stream))
     else:
         _call("dit_qk_rmsnorm_rope_ex", *args, mode, _stream(stream))
+
+
+def _offsets(pos_offset: torch.Tensor, B: int) -> int:
+    if pos_offset.dtype != torch.int32 or not pos_offset.is_cuda or not pos_offset.is_contiguous() or \
+            tuple(pos_offset.shape) != (B,):
+        raise TypeError("pos_offset: expected a contiguous int32 CUDA vector [num_seqs]")
+    return pos_offset.data_ptr() or None
 
 
 def dit_adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
@@ -327,13 +341,15 @@ def dit_validate_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tens
 
 
 def dit_av_stream_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Tensor, rope_grid: torch.Tensor,
-                          *, out: Optional[tuple] = None, stream=None) -> tuple:
+                          *, pos_offset: Optional[torch.Tensor] = None, out: Optional[tuple] = None,
+                          stream=None) -> tuple:
     """Per-stream descriptor of joint audio-video sequences: sequence b becomes
     sequences 2b (its T*H*W video rows) and 2b + 1 (its audio rows and
     padding).  Returns (cu_seqlens_av, cu_seqlens_padded_av), int32
     [2 * num_seqs + 1] on the device.  Pass them to the modulated ops with
     vectors laid out [num_seqs, 2, ...] viewed as [2 * num_seqs, ...], e.g. for
-    mod [B, 2, 6, C]: shift = mod.view(2 * B, 6, C)[:, 0]."""
+    mod [B, 2, 6, C]: shift = mod.view(2 * B, 6, C)[:, 0].  pos_offset: as in
+    dit_qk_rmsnorm_rope, for one rank's slice of longer sequences."""
     cs, cp, B = _packing(cu_seqlens, cu_seqlens_padded)
     if rope_grid.dtype != torch.int32 or not rope_grid.is_cuda or not rope_grid.is_contiguous() or \
             tuple(rope_grid.shape) != (B, 3):
@@ -344,8 +360,9 @@ def dit_av_stream_seqlens(cu_seqlens: torch.Tensor, cu_seqlens_padded: torch.Ten
     for t in out:
         if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != 2 * B + 1:
             raise TypeError(f"out: expected two contiguous int32 CUDA vectors of {2 * B + 1} entries")
-    _call("dit_av_stream_seqlens", cs, cp, rope_grid.data_ptr(), B, out[0].data_ptr(), out[1].data_ptr(),
-          _stream(stream))
+    po = None if pos_offset is None else _offsets(pos_offset, B)
+    _call("dit_av_stream_seqlens", cs, cp, rope_grid.data_ptr() or None, po, B, out[0].data_ptr(),
+          out[1].data_ptr(), _stream(stream))
     return out
 
 

@@ -85,6 +85,21 @@ dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k, int64_
                                   const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
                                   float rope_theta, float eps, int32_t rope_mode, void* stream)
 {
+    return dit_qk_rmsnorm_rope_shard(q, q_row_stride, k, k_row_stride, q_weight, k_weight, cu_seqlens,
+                                     cu_seqlens_padded, num_seqs, num_rows_padded, num_q_heads, num_k_heads,
+                                     head_dim, rope_grid, sec_t, sec_h, sec_w, rope_theta, eps, rope_mode, nullptr,
+                                     stream);
+}
+
+dit_status dit_qk_rmsnorm_rope_shard(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                                     const void* q_weight, const void* k_weight,
+                                     const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                     int32_t num_seqs, int64_t num_rows_padded,
+                                     int32_t num_q_heads, int32_t num_k_heads, int32_t head_dim,
+                                     const int32_t* rope_grid, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+                                     float rope_theta, float eps, int32_t rope_mode, const int32_t* pos_offset,
+                                     void* stream)
+{
     bool empty = false;
     dit_status st = check_packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded, &empty);
     if (st != DIT_OK)
@@ -110,7 +125,8 @@ dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k, int64_
         return DIT_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(q_weight) || !aligned16(k_weight) ||
         !mult8(q_row_stride) || !mult8(k_row_stride) ||
-        (rope_grid && (reinterpret_cast<uintptr_t>(rope_grid) & 3u)))
+        (rope_grid && (reinterpret_cast<uintptr_t>(rope_grid) & 3u)) ||
+        (pos_offset && (reinterpret_cast<uintptr_t>(pos_offset) & 3u)))
         return DIT_ERR_ALIGN;
 
     dit::QkParams p{};
@@ -119,6 +135,7 @@ dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k, int64_
     p.q_weight = static_cast<const uint16_t*>(q_weight);
     p.k_weight = static_cast<const uint16_t*>(k_weight);
     p.rope_grid = rope_mode == DIT_ROPE_NONE ? nullptr : rope_grid;
+    p.pos_offset = rope_mode == DIT_ROPE_NONE ? nullptr : pos_offset;
     p.q_row_stride = q_row_stride;
     p.k_row_stride = k_row_stride;
     p.pk = packing(cu_seqlens, cu_seqlens_padded, num_seqs, num_rows_padded);
@@ -342,8 +359,8 @@ dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seq
 }
 
 dit_status dit_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
-                                 const int32_t* rope_grid, int32_t num_seqs, int32_t* out_cu_seqlens,
-                                 int32_t* out_cu_seqlens_padded, void* stream)
+                                 const int32_t* rope_grid, const int32_t* pos_offset, int32_t num_seqs,
+                                 int32_t* out_cu_seqlens, int32_t* out_cu_seqlens_padded, void* stream)
 {
     if (num_seqs < 0 || num_seqs > (INT32_MAX - 1) / 2)
         return DIT_ERR_SHAPE;
@@ -351,11 +368,12 @@ dit_status dit_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_se
         (num_seqs > 0 && !rope_grid))
         return DIT_ERR_NULL;
     const uintptr_t any = reinterpret_cast<uintptr_t>(cu_seqlens) | reinterpret_cast<uintptr_t>(cu_seqlens_padded) |
-                          reinterpret_cast<uintptr_t>(rope_grid) | reinterpret_cast<uintptr_t>(out_cu_seqlens) |
+                          reinterpret_cast<uintptr_t>(rope_grid) | reinterpret_cast<uintptr_t>(pos_offset) |
+                          reinterpret_cast<uintptr_t>(out_cu_seqlens) |
                           reinterpret_cast<uintptr_t>(out_cu_seqlens_padded);
     if (any & 3u)
         return DIT_ERR_ALIGN;
-    return from_cuda(dit::launch_av_stream_seqlens(cu_seqlens, cu_seqlens_padded, rope_grid, num_seqs,
+    return from_cuda(dit::launch_av_stream_seqlens(cu_seqlens, cu_seqlens_padded, rope_grid, pos_offset, num_seqs,
                                                    out_cu_seqlens, out_cu_seqlens_padded,
                                                    static_cast<cudaStream_t>(stream)));
 }

@@ -28,6 +28,7 @@ struct QkParams {
     const uint16_t* q_weight;
     const uint16_t* k_weight;
     const int32_t* rope_grid;
+    const int32_t* pos_offset;  // [num_seqs] start of each sequence's rows in the whole sequence, or null
     int64_t q_row_stride;
     int64_t k_row_stride;
     Packing pk;
@@ -115,8 +116,8 @@ cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream);
 cudaError_t launch_swiglu(const SwigluParams& p, cudaStream_t stream);
 cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream);
 cudaError_t launch_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
-                                     const int32_t* rope_grid, int32_t num_seqs, int32_t* out_cu_seqlens,
-                                     int32_t* out_cu_seqlens_padded, cudaStream_t stream);
+                                     const int32_t* rope_grid, const int32_t* pos_offset, int32_t num_seqs,
+                                     int32_t* out_cu_seqlens, int32_t* out_cu_seqlens_padded, cudaStream_t stream);
 cudaError_t launch_validate_seqlens(const Packing& pk, int64_t num_rows_padded, int32_t* flag,
                                     cudaStream_t stream);
 

@@ -204,21 +204,24 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         // Positions of this row: a row inside the sequence's T x H x W video
         // grid (t-major, then h, then w) is 3D; every later row is 1D, counted
         // from the end of the grid.  Without a grid every row is 1D.
+        // g: the row's index in its whole sequence (the buffer may hold one
+        // rank's slice of it, starting at row pos_offset[seq])
+        const long long g = (long long)s.local + (p.pos_offset != nullptr ? __ldg(p.pos_offset + s.seq) : 0);
         bool is3d = false;
         long long pt = 0, ph = 0, pw = 0;
-        long long pos1 = s.local;
+        long long pos1 = g;
         if (p.rope_grid != nullptr) {
             const long long T = __ldg(p.rope_grid + 3 * s.seq);
             const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
             const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
             const long long thw = T * H * W;
-            if (s.local < thw) {
+            if (g < thw) {
                 is3d = true;
-                pt = s.local / (H * W);
-                ph = (s.local / W) % H;
-                pw = s.local % W;
+                pt = g / (H * W);
+                ph = (g / W) % H;
+                pw = g % W;
             } else {
-                pos1 = s.local - thw;
+                pos1 = g - thw;
             }
         }
 #pragma unroll

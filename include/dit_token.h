@@ -128,6 +128,24 @@ DIT_API dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k
                                           int32_t sec_w, float rope_theta, float eps, int32_t rope_mode,
                                           void* stream);
 
+/* dit_qk_rmsnorm_rope_ex on one rank's slice of longer sequences.
+ *
+ * Pages: first page "Key takeaways" bullet 1 (each rank's rotary work is
+ * restricted to its own rows of the packed sequence).  The rows of sequence b
+ * in this buffer are rows pos_offset[b], pos_offset[b] + 1, ... of the whole
+ * sequence b, and take that sequence's positions: with rope_grid[b] =
+ * (T, H, W), whole-sequence rows below T*H*W are 3D, the rest 1D counted from
+ * the end of the grid.  pos_offset: device int32 [num_seqs] (>= 0), or NULL
+ * (every offset 0: the _ex call).  Ignored when rope_mode is DIT_ROPE_NONE. */
+DIT_API dit_status dit_qk_rmsnorm_rope_shard(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
+                                             const void* q_weight, const void* k_weight,
+                                             const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
+                                             int32_t num_seqs, int64_t num_rows_padded, int32_t num_q_heads,
+                                             int32_t num_k_heads, int32_t head_dim, const int32_t* rope_grid,
+                                             int32_t sec_t, int32_t sec_h, int32_t sec_w, float rope_theta,
+                                             float eps, int32_t rope_mode, const int32_t* pos_offset,
+                                             void* stream);
+
 /* Adaptive LayerNorm modulation: out = LN(x) * (1 + scale_b) + shift_b.
  *
  * Pages: first page "Key takeaways" bullet 2 (the modulation and the
@@ -283,13 +301,18 @@ DIT_API dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t
  * audio set to audio rows.  RoPE keeps the original descriptor (positions are
  * per request).
  *
+ * For one rank's slice of longer sequences (pos_offset[b] = the whole-sequence
+ * index of b's first row, as in dit_qk_rmsnorm_rope_shard) v_b counts the grid
+ * rows past that start: clamp(T*H*W - pos_offset[b], 0, min(L_b, padded_b)).
+ *
  * cu_seqlens, cu_seqlens_padded  device int32 [num_seqs + 1]
  * rope_grid                      device int32 [num_seqs][3] (may be NULL only if num_seqs == 0)
+ * pos_offset                     device int32 [num_seqs], or NULL (all 0)
  * out_cu_seqlens, out_cu_seqlens_padded  device int32 [2 * num_seqs + 1], written
  * One small kernel on `stream`; no synchronization.  Entries 0 are copied. */
 DIT_API dit_status dit_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
-                                         const int32_t* rope_grid, int32_t num_seqs, int32_t* out_cu_seqlens,
-                                         int32_t* out_cu_seqlens_padded, void* stream);
+                                         const int32_t* rope_grid, const int32_t* pos_offset, int32_t num_seqs,
+                                         int32_t* out_cu_seqlens, int32_t* out_cu_seqlens_padded, void* stream);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 DIT_API const char* dit_status_string(dit_status s);

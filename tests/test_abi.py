@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
-    assert len(names) == 15, names
+    assert len(names) == 16, names
     for n in names:
         assert hasattr(L, n), n
     assert L.dit_abi_version() == 1
@@ -173,12 +173,25 @@ def test_modulation_dtype_entries(L):
 
 def test_av_stream_seqlens_argument_checks(L):
     f = L.dit_av_stream_seqlens
-    assert f(P, P, P, -1, P, P, None) == SHAPE
-    assert f(P, P, P, 1 << 30, P, P, None) == SHAPE
-    assert f(None, P, P, 2, P, P, None) == NULL
-    assert f(P, P, None, 2, P, P, None) == NULL        # the split needs the grid
-    assert f(P, P, P, 2, P, None, None) == NULL
-    assert f(P, P, P + 2, 2, P, P, None) == ALIGN
+    assert f(P, P, P, None, -1, P, P, None) == SHAPE
+    assert f(P, P, P, None, 1 << 30, P, P, None) == SHAPE
+    assert f(None, P, P, None, 2, P, P, None) == NULL
+    assert f(P, P, None, None, 2, P, P, None) == NULL        # the split needs the grid
+    assert f(P, P, P, None, 2, P, None, None) == NULL
+    assert f(P, P, P + 2, None, 2, P, P, None) == ALIGN
+    assert f(P, P, P, P + 2, 2, P, P, None) == ALIGN
+
+
+def test_qk_shard_argument_checks(L):
+    def sh(po, **kw):
+        a = dict(q=P, B=1, mode=0)
+        a.update(kw)
+        return L.dit_qk_rmsnorm_rope_shard(a["q"], 256, P, 256, P, P, P, P, a["B"], 16, 2, 2, 128, None, 0, 0, 0,
+                                           10000.0, 1e-6, a["mode"], po, None)
+    assert sh(P + 2) == ALIGN
+    assert sh(None, q=None) == NULL
+    assert sh(P, mode=7) == UNSUP
+    assert sh(P + 2, B=0) == OK          # empty batch: nothing checked past the shapes
 
 
 def test_frames_argument_checks(L):

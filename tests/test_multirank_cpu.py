@@ -1,6 +1,8 @@
-"""Host logic of the multi-GPU benchmark path, on CPU with two gloo ranks:
-each rank draws its own batch of the same shapes (no data is exchanged), the
-timing is the max over ranks, and every rank takes the same collective steps."""
+"""Host logic of the multi-GPU paths, on CPU with two gloo ranks: in the
+benchmark each rank draws its own batch of the same shapes (no data is
+exchanged), the timing is the max over ranks, and every rank takes the same
+collective steps; when ranks split one batch instead, each rank's slice
+(with its rows' whole-sequence positions) gives the unsharded result."""
 import os
 import socket
 
@@ -59,3 +61,54 @@ def test_single_process_needs_no_process_group():
     import bench
     assert bench.reduce_max(3.5, torch.device("cpu")) == 3.5
     assert bench.data_seed(5, 0) == 5 and bench.data_seed(5, 1) != 5
+
+
+def _shard_worker(rank, world, port, out):
+    """One rank's slice of one batch: the rank runs the oracle on its own rows
+    (with their whole-sequence positions) and the slices are gathered."""
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from dit_token_b200 import workloads as W
+    from dit_token_b200.shard import shard_packing
+    from _util import tbits
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = W.custom("sp", (700, 45, 300), (704, 48, 304), hidden=128, num_q_heads=2, num_k_heads=1,
+                     head_dim=64, inner=64, grids=((4, 6, 25), (0, 0, 0), (3, 5, 10)), sections=(24, 20, 20))
+        inp = W.qk_inputs(w)
+        q, k = tbits(W.rows_view(inp["q"])), tbits(W.rows_view(inp["k"]))
+        sh = shard_packing(w.cu_seqlens, w.cu_seqlens_padded, w.rope_grid, rank, world)
+        qo, ko = oracle.qk_rmsnorm_rope(q[sh.rows], k[sh.rows], tbits(inp["q_weight"]), tbits(inp["k_weight"]),
+                                        sh.cu_seqlens, sh.cu_seqlens_padded, num_q_heads=2, num_k_heads=1,
+                                        head_dim=64, rope_grid=sh.rope_grid, sections=w.sections,
+                                        pos_offset=sh.pos_offset)
+        mine = torch.from_numpy(np.concatenate([qo.astype(np.int64), ko.astype(np.int64)], axis=1))
+        sizes = [torch.zeros(1, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(sizes, torch.tensor([mine.shape[0]]))
+        biggest = int(max(s.item() for s in sizes))
+        padded = torch.zeros(biggest, mine.shape[1], dtype=torch.int64)
+        padded[: mine.shape[0]] = mine
+        parts = [torch.zeros_like(padded) for _ in range(world)]
+        dist.all_gather(parts, padded)
+        if rank == 0:
+            got = np.concatenate([p[: int(n.item())].numpy() for p, n in zip(parts, sizes)])
+            fq, fk = oracle.qk_rmsnorm_rope(q, k, tbits(inp["q_weight"]), tbits(inp["k_weight"]), w.cu_seqlens,
+                                            w.cu_seqlens_padded, num_q_heads=2, num_k_heads=1, head_dim=64,
+                                            rope_grid=w.rope_grid, sections=w.sections)
+            want = np.concatenate([fq.astype(np.int64), fk.astype(np.int64)], axis=1)
+            valid = w.valid_rows()
+            out["equal"] = bool(np.array_equal(got[valid], want[valid]))
+            out["rows"] = got.shape[0] == want.shape[0]
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_split_one_batch_with_global_positions():
+    mgr = mp.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    mp.spawn(_shard_worker, args=(2, port, out), nprocs=2, join=True)
+    assert out["rows"] and out["equal"]
