@@ -80,11 +80,11 @@ def _code_only(text: str) -> str:
 
 
 def kernel_source_digest(op: str) -> str:
-    """Digest of the code of an op's kernel file, the shared device header and
-    the launch header (comments and layout ignored)."""
+    """Digest of the code of an op's kernel file and of the shared device
+    header (comments and layout ignored)."""
     csrc = os.path.join(ROOT, "dit_token_b200", "csrc")
     h = hashlib.sha256()
-    for name in (f"{op}.cu", "common.cuh", "launch.h"):
+    for name in (f"{op}.cu", "common.cuh"):
         with open(os.path.join(csrc, name)) as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
