@@ -100,3 +100,20 @@ def test_offset_zero_is_the_plain_call():
     b = run_all(x, y, mod, cs, cp, GRID, np.zeros(len(LENGTHS), np.int32), C)
     for name in a:
         assert np.array_equal(a[name], b[name]), name
+
+
+def test_more_ranks_than_tokens_and_empty_batches():
+    cs, cp = cu([2, 0, 1]), cu([8, 8, 8])
+    shards = [shard_packing(cs, cp, None, r, 8) for r in range(8)]
+    assert sum(s.num_valid for s in shards) == 3
+    assert np.array_equal(np.concatenate([s.rows for s in shards]), np.arange(24))
+    assert all(s.rope_grid is None for s in shards)
+    for s in shards:                                   # every shard is a well-formed packing
+        assert s.cu_seqlens[0] == 0 and s.cu_seqlens_padded[0] == 0
+        assert np.all(np.diff(s.cu_seqlens) <= np.diff(s.cu_seqlens_padded))
+        assert s.cu_seqlens_padded[-1] == s.num_rows_padded
+    empty = [shard_packing(cu([0, 0]), cu([4, 4]), None, r, 3) for r in range(3)]
+    assert [e.num_seqs for e in empty] == [0, 0, 2]    # padding-only sequences go to the last rank
+    assert np.array_equal(empty[2].rows, np.arange(8))
+    with pytest.raises(ValueError):
+        shard_packing(cs, cp, None, 3, 3)
