@@ -35,8 +35,10 @@
 // of DRAM peak, SM activity very uneven -- active cycles min / mean / max
 // 2k / 132k / 203k of 210k -- with the copy engine's pipe nearly idle); this
 // kernel with each register vector refilled with the next row's during the
-// output pass 248 us against 244 us without (both with a clean L2); this
-// kernel 244-264 us.
+// output pass 248 us against 244 us without (both with a clean L2); the
+// next row (or the one after) pulled into L2 by a 1-D bulk prefetch
+// (cp.async.bulk.prefetch.L2) issued by one lane per row 260 / 303 us against
+// 242 us; this kernel 242-264 us.
 #include "common.cuh"
 #include "launch.h"
 
