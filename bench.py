@@ -333,11 +333,20 @@ def time_e2e(sets, steps: int, warmup: int, device):
     downloads its outputs, all inside the timed region.  Uploads, kernels and
     downloads run on three streams ordered by events, so the two copy
     directions overlap each other and the kernels; two device buffer sets
-    alternate between steps (q and k are updated in place)."""
-    h_in = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_inputs(op)]
-            for op in OPS}
-    h_out = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_outputs(op)]
-             for op in OPS}
+    alternate between steps (q and k are updated in place).  Returns None on
+    every rank when any rank cannot pin its host buffers."""
+    try:
+        h_in = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_inputs(op)]
+                for op in OPS}
+        h_out = {op: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0].op_outputs(op)]
+                 for op in OPS}
+        pinned = 1.0
+    except RuntimeError:  # the host could not pin the step's buffers
+        h_in = h_out = None
+        pinned = 0.0
+    # every rank takes the same collective steps: all time the leg, or none does
+    if reduce_max(1.0 - pinned, torch.device("cuda", torch.cuda.current_device())) > 0.0:
+        return None
     for op in OPS:
         for h, d in zip(h_in[op], sets[0].op_inputs(op)):
             h.copy_(d)
@@ -496,12 +505,20 @@ def run_dit(args):
     next_ms = {k: reduce_max(v, device)
                for k, v in time_next_ops(step, args.steps, args.warmup, device, args.scale).items()}
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    # two device buffer sets let consecutive end-to-end steps overlap; one step needs one
     # two device buffer sets let consecutive end-to-end steps overlap; the
     # small profiling-size runs (--scale < 1) keep one to stay small
     sets = [step, Step(w, host, device)] if args.scale >= 1.0 else [step]
-    e2e_ms, h2d, d2h = time_e2e(sets, e2e_steps, min(args.warmup, 3), device)
-    e2e_max = reduce_max(e2e_ms, device)
+    timed_e2e = time_e2e(sets, e2e_steps, min(args.warmup, 3), device)
+    if timed_e2e is None:
+        e2e = {"value": None, "unit": UNIT,
+               "unavailable": "the host could not pin the step's input and output buffers on every rank"}
+    else:
+        e2e_ms, h2d, d2h = timed_e2e
+        e2e_max = reduce_max(e2e_ms, device)
+        e2e = {"value": round(w.num_valid * world * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": round(e2e_max / e2e_steps, 3),
+               "schedule": "per-op upload / kernel / download on 3 streams, 2 device buffer sets"}
 
     tokens = w.num_valid * world
     value = tokens * args.steps / (max_ms / 1e3)
@@ -541,10 +558,7 @@ def run_dit(args):
                 "gbs": round(5 * math.prod(frames_shape(args.scale)) / (next_ms["frames_to_u8"] / 1e3) / 1e9, 1),
                 "bytes": 5 * math.prod(frames_shape(args.scale))},
         },
-        "e2e": {"value": round(tokens * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "ms_per_step": round(e2e_max / e2e_steps, 3),
-                "schedule": "per-op upload / kernel / download on 3 streams, 2 device buffer sets"},
+        "e2e": e2e,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
