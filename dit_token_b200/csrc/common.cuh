@@ -124,25 +124,11 @@ __device__ __forceinline__ void st_stream(uint16_t* p, uint4 v)
     __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
-__device__ __forceinline__ uint4 ld_shared_vec(const uint16_t* p)
+// 8 elements of a small vector that many rows share (norm weights, gates,
+// shifts, scales): read-only path, kept in L1/L2.
+__device__ __forceinline__ uint4 ld_readonly(const uint16_t* p)
 {
     return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
-// Asynchronous 16-byte global -> shared copies (L1 bypassed), completed with
-// commit/wait groups: a hardware wait, no polling loop.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
-{
-    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------ bf16 <-> fp32

@@ -243,8 +243,8 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         unpack8(make_uint4(q0.x, q0.y, q1.x, q1.y), wq);
         unpack8(make_uint4(k0.x, k0.y, k1.x, k1.y), wk);
     } else {
-        unpack8(ld_shared_vec(p.q_weight + 8 * li), wq);
-        unpack8(ld_shared_vec(p.k_weight + 8 * li), wk);
+        unpack8(ld_readonly(p.q_weight + 8 * li), wq);
+        unpack8(ld_readonly(p.k_weight + 8 * li), wk);
     }
     PairCoef pq{}, pk{};
     if (MODE != kRopeNone) {
