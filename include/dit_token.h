@@ -15,13 +15,15 @@
  *
  * Common conventions
  * ------------------
- * Data type   every activation, weight and modulation vector is bf16
- *             (IEEE binary32 upper half), row-major; arithmetic is fp32 and
- *             every output element is rounded once, to nearest-even.
+ * Data type   every activation and weight is bf16 (IEEE binary32 upper
+ *             half), row-major; modulation vectors are bf16, or fp32 through
+ *             the _ex entry points; decoded frames are fp32.  Arithmetic is
+ *             fp32 and every output element is rounded once, to
+ *             nearest-even.
  * Pointers    all tensor pointers are DEVICE pointers, owned by the caller;
  *             they must be 16-byte aligned.  Strides are in ELEMENTS and must
- *             be multiples of 8 (16 bytes); so must hidden, inner and
- *             head_dim.
+ *             be multiples of 8 (16 bytes; fp32 vector strides multiples of
+ *             4); so must hidden, inner and head_dim.
  * Packing     cu_seqlens[num_seqs+1] (device, int32): cumulative VALID lengths,
  *             cu_seqlens[0] = 0.  cu_seqlens_padded[num_seqs+1] (device,
  *             int32): first padded row of every sequence, the last entry the
@@ -34,7 +36,8 @@
  *             skipped.  dit_validate_seqlens checks them on the device.
  * Aliasing    in-place use is allowed only as exact aliasing (same pointer
  *             and stride): out == x for dit_adaln_modulate and
- *             dit_gated_residual; q and k are always updated in place.
+ *             dit_gated_residual, res_out == x for dit_gated_residual_adaln;
+ *             q and k are always updated in place.
  *             Partial overlap is undefined.
  * Stream      `stream` is a cudaStream_t (NULL = the legacy default stream).
  *             Calls only enqueue work: they never synchronize, allocate or
