@@ -165,18 +165,20 @@ cudaError_t launch_team(const FusedParams& p, int vpt, cudaStream_t stream)
 
 }  // namespace
 
-// Team size: the smallest of 1, 2, 4, 8 warps that holds the row in at most 8
-// vectors per lane (hidden 2048 -> 1 warp, 3072 -> 2, 5120 -> 4).
+// Team size: the smallest of 2, 4, 8 warps that holds the row in at most 8
+// vectors per lane (hidden 2048 -> 2 warps, 3072 -> 2, 5120 -> 4).  A single
+// warp per row was measured slower on short rows (hidden 2048: 36.9 against
+// 29.9 us for 8192 rows), and at most 4 vectors per lane slower on long ones
+// (hidden 5120: 568 against 456 us).
 cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream)
 {
     const int nvec = p.hidden / 8;
-    for (int team = 1; team <= kWarpsPerCta; team *= 2) {
+    for (int team = 2; team <= kWarpsPerCta; team *= 2) {
         const int per = team * kWarp;
         const int vpt = (nvec + per - 1) / per;
         if (vpt > 8)
             continue;
         switch (team) {
-        case 1: return launch_team<1>(p, vpt, stream);
         case 2: return launch_team<2>(p, vpt, stream);
         case 4: return launch_team<4>(p, vpt, stream);
         default: return launch_team<8>(p, vpt, stream);
