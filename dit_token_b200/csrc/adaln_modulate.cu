@@ -326,6 +326,12 @@ cudaError_t launch_adaln_modulate(const AdalnParams& p, cudaStream_t stream)
 {
     const int nvec = p.hidden / 8;
     const int vpt = (nvec + kWarp - 1) / kWarp;
+    // Rows of 2304-3072 elements with bf16 vectors: two warps per row measured
+    // faster than one (hidden 3072: 61,888 rows 129.2 against 135.4 us, 16,256
+    // rows 41.0 against 42.3 us); with fp32 vectors, and at other widths
+    // (2048: 22.6 against 21.5 us; 5120: 268.9 against 243.9 us), slower.
+    if (!p.mod_f32 && vpt > 8 && vpt <= 12)
+        return launch_team<2>(p, stream);
     if (vpt <= kMaxWarpVpt) {
         switch (vpt) {
         case 1: return launch_warp<1>(p, stream);
