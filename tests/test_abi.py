@@ -1,7 +1,6 @@
 """C-ABI checks that need no GPU: the library loads, exports every entry point
 the header declares, and rejects bad arguments with the documented status
 before launching anything."""
-import ctypes
 import os
 import re
 

@@ -13,7 +13,6 @@ import torch
 import dit_token_b200 as dit
 from dit_token_b200 import workloads as W
 import _parity as P
-from _util import tbits
 
 pytestmark = pytest.mark.gpu
 

@@ -7,7 +7,6 @@ compared element by element (the oracle computes those rows one by one);
 every padding row and the canary rows around each buffer are checked
 bit-exactly at full size, and a second run must be bitwise identical.
 """
-import numpy as np
 import pytest
 import torch
 
