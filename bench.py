@@ -24,6 +24,11 @@ bandwidth; ``cpu_baseline`` times the plain CPU oracle on a bounded sample.
 ``--impl reference`` times the CPU oracle alone (the only reference this
 operator set has): rank 0 runs K + W bounded samples of the same workload on
 the host cores and prints the same JSON line with "impl": "reference".
+
+``--table`` prints a per-op markdown table over every workload and
+``--variants`` one over the operator variants (fp32 and per-stream
+modulation vectors, rotary layouts, grouped K heads, head_dim 256), both
+with a read-only pass over 512 MB before every timed launch (clean L2).
 """
 from __future__ import annotations
 
