@@ -332,6 +332,35 @@ def time_device(step: Step, steps: int, warmup: int, device):
     return elapsed_ms, op_ms, (t_host0, t_host1)
 
 
+def time_graph(step: Step, steps: int, warmup: int, device) -> float:
+    """The same step captured once in a CUDA graph and replayed `steps` times
+    (the library's calls only enqueue work, so they capture as they are):
+    mean ms per replay, for comparison with the eagerly launched step."""
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step.run()  # warm the launch paths on the capture stream
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step.run()
+    for _ in range(warmup):
+        graph.replay()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(device)
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    end.record()
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = start.elapsed_time(end) / steps
+    del graph
+    return ms
+
+
 def time_e2e(sets, steps: int, warmup: int, device):
     """The same step through the public API for a caller whose data lives in
     pinned host memory: every step uploads each op's inputs, runs the op and
@@ -509,6 +538,7 @@ def run_dit(args):
     op_ms_max = {op: reduce_max(v, device) for op, v in op_ms.items()}
     next_ms = {k: reduce_max(v, device)
                for k, v in time_next_ops(step, args.steps, args.warmup, device, args.scale).items()}
+    graph_ms = reduce_max(time_graph(step, args.steps, args.warmup, device), device)
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     # two device buffer sets let consecutive end-to-end steps overlap; the
     # small profiling-size runs (--scale < 1) keep one to stay small
@@ -564,6 +594,8 @@ def run_dit(args):
                 "bytes": 5 * math.prod(frames_shape(args.scale))},
         },
         "e2e": e2e,
+        "graph": {"ms_per_step": round(graph_ms, 4), "steps": args.steps,
+                  "note": "the same step captured once in a CUDA graph and replayed; value uses the eager step"},
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
