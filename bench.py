@@ -702,8 +702,9 @@ def run_table(args):
 def run_variants(args):
     """Markdown table of the operator variants (fp32 and per-stream modulation
     vectors, rotary layouts, grouped K heads, head_dim 256) on the batched
-    varlen and long video workloads, timed like --table (L2 evicted before
-    every launch, median of --steps launches)."""
+    varlen and long video workloads, and of Q/K normalization and SwiGLU at
+    VAE-like shapes, timed like --table (L2 evicted before every launch,
+    median of --steps launches)."""
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     from dit_token_b200 import build
@@ -775,6 +776,26 @@ def run_variants(args):
                     rope_theta=w.rope_theta, eps=w.eps, rope_mode=mode)), 8 * C * n, n)
         del step, mods, m32, mav
         torch.cuda.empty_cache()
+
+    # VAE-like shapes (the pages reuse the fused Q/K norm and SwiGLU in the VAE
+    # decoder and give no shapes): one sequence of 2^20 tokens, 512 channels as
+    # 8 heads of 64 without rotation, SwiGLU inner 512.  Values N(0, 1) drawn on
+    # the device (only the timing is of interest here).
+    n = 1 << 20
+    gen = torch.Generator(device=device).manual_seed(args.seed)
+    cs = torch.tensor([0, n], dtype=torch.int32, device=device)
+    q = torch.randn(n, 512, generator=gen, device=device).to(torch.bfloat16)
+    k = torch.randn(n, 512, generator=gen, device=device).to(torch.bfloat16)
+    w64 = torch.ones(64, dtype=torch.bfloat16, device=device)
+    row("vae 1x1048576", "qk_rmsnorm_rope", "none pairs, 8x64", timed(lambda: dit.dit_qk_rmsnorm_rope(
+        q, k, w64, w64, cs, cs, num_q_heads=8, num_k_heads=8, head_dim=64, rope_mode="none")), 8 * 512 * n, n)
+    del q, k
+    ab = torch.randn(n, 1024, generator=gen, device=device).to(torch.bfloat16)
+    out = torch.empty(n, 512, dtype=torch.bfloat16, device=device)
+    row("vae 1x1048576", "swiglu", "inner 512", timed(lambda: dit.dit_swiglu(
+        ab[:, :512], ab[:, 512:], cs, cs, out=out)), 6 * 512 * n, n)
+    del ab, out
+    torch.cuda.empty_cache()
 
 
 def main(argv=None):

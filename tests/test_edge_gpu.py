@@ -248,3 +248,19 @@ def test_gqa_at_scale_and_thousands_of_sequences():
     padded = [int(L) + int(rng.integers(0, 3)) for L in lengths]
     w = W.custom("many2", lengths, padded, hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64, seed=3)
     all_ops_full(w)
+
+
+def test_vae_like_shapes():
+    """Q/K normalization without rotation and SwiGLU at VAE-like shapes: one
+    sequence of 2^18 tokens, 512 channels as 8 heads of 64, SwiGLU inner 512."""
+    n = 1 << 18
+    w = W.custom("vae", (n,), (n,), hidden=512, num_q_heads=8, num_k_heads=8, head_dim=64, inner=512, seed=4)
+    rows = W.sample_rows(w, per_seq=2000)
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp, rope_mode="none")
+    qo, ko = P.oracle_qk(w, inp, rows, rope_mode="none")
+    P.assert_close(P.gather_rows(q, rows), qo[rows], "vae q")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], "vae k")
+    sw = W.swiglu_inputs(w)
+    out = P.gpu_swiglu(w, sw)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, sw, rows)[rows], "vae swiglu")
