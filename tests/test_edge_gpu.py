@@ -264,3 +264,42 @@ def test_vae_like_shapes():
     sw = W.swiglu_inputs(w)
     out = P.gpu_swiglu(w, sw)
     P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, sw, rows)[rows], "vae swiglu")
+
+
+@pytest.mark.parametrize("mode", ["interleaved", "half"])
+@pytest.mark.parametrize("sliced", [False, True])
+def test_small_rows_several_per_warp(mode, sliced):
+    """Rows of 256 bytes (one q and one k head of 64) in the tens of
+    thousands: each warp takes several rows, its head batches pipelined across
+    row boundaries.  Ragged 3D grids with 1D tails, empty sequences, and (when
+    sliced) per-sequence position offsets, all against the oracle."""
+    rng = np.random.default_rng(21 if sliced else 20)
+    B = 160
+    lengths = rng.integers(0, 400, B)
+    lengths[::37] = 0
+    padded = lengths + rng.integers(0, 9, B)
+    grids = np.stack([rng.integers(0, 4, B), rng.integers(1, 7, B), rng.integers(1, 9, B)], axis=1)
+    w = W.custom("small", lengths, padded, hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64,
+                 grids=grids, sections=(24, 20, 20), seed=9)
+    assert w.num_valid > 4 * 32 * 148          # enough rows that the launcher puts several on a warp
+    po = rng.integers(0, 60, B).astype(np.int32) if sliced else None
+    inp = W.qk_inputs(w)
+    cs, cp, grid = P.device_packing(w)
+    q, k = inp["q"].cuda(), inp["k"].cuda()
+    dit.dit_qk_rmsnorm_rope(W.rows_view(q), W.rows_view(k), inp["q_weight"].cuda(), inp["k_weight"].cuda(), cs, cp,
+                            num_q_heads=1, num_k_heads=1, head_dim=64, rope_grid=grid, sections=w.sections,
+                            rope_theta=w.rope_theta, eps=w.eps, rope_mode=mode,
+                            pos_offset=None if po is None else torch.from_numpy(po).cuda())
+    rows = w.valid_rows()
+    import oracle
+    from _util import tbits
+    qo, ko = oracle.qk_rmsnorm_rope(tbits(W.rows_view(inp["q"])), tbits(W.rows_view(inp["k"])),
+                                    tbits(inp["q_weight"]), tbits(inp["k_weight"]), w.cu_seqlens,
+                                    w.cu_seqlens_padded, num_q_heads=1, num_k_heads=1, head_dim=64,
+                                    rope_grid=w.rope_grid, sections=w.sections, rope_theta=w.rope_theta,
+                                    eps=w.eps, rope_mode=mode, pos_offset=po)
+    P.assert_close(P.gather_rows(q, rows), qo[rows], f"small rows q {mode}")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], f"small rows k {mode}")
+    keep = P.untouched_rows(w)
+    P.assert_untouched(q, inp["q"], keep, "small rows q")
+    P.assert_untouched(k, inp["k"], keep, "small rows k")
