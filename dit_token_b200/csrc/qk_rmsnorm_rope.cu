@@ -168,64 +168,12 @@ __device__ __forceinline__ void rms_rotate_batch(uint16_t* row, int H, int h0, i
     }
 }
 
-// The per-row setup of the rotation: the row's positions (3D inside its
-// sequence's grid, 1D after it, offset by the sequence's slice start), the
-// lane's 4 cos/sin pairs, and the weights folded into the coefficients.
-template <int D, int MODE>
-__device__ __forceinline__ void row_coefficients(const QkParams& p, int seq, int local, int li, const float (&wq)[8],
-                                                 const float (&wk)[8], PairCoef& pq, PairCoef& pk)
-{
-    if (MODE == kRopeNone)
-        return;
-    // g: the row's index in its whole sequence (the buffer may hold one
-    // rank's slice of it, starting at row pos_offset[seq])
-    const long long g = (long long)local + (p.pos_offset != nullptr ? __ldg(p.pos_offset + seq) : 0);
-    // Positions: a row inside the sequence's T x H x W video grid (t-major,
-    // then h, then w) is 3D; every later row is 1D, counted from the end of
-    // the grid.  Without a grid every row is 1D.
-    bool is3d = false;
-    long long pt = 0, ph = 0, pw = 0;
-    long long pos1 = g;
-    if (p.rope_grid != nullptr) {
-        const long long T = __ldg(p.rope_grid + 3 * seq);
-        const long long H = __ldg(p.rope_grid + 3 * seq + 1);
-        const long long W = __ldg(p.rope_grid + 3 * seq + 2);
-        const long long thw = T * H * W;
-        if (g < thw) {
-            is3d = true;
-            pt = g / (H * W);
-            ph = (g / W) % H;
-            pw = g % W;
-        } else {
-            pos1 = g - thw;
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int j = 4 * li + e;
-        const int ax = p.axis[j];
-        const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
-        const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
-        float c, sv;
-        pair_cos_sin(ang, c, sv);
-        int a, b;
-        pair_regs<MODE>(e, a, b);
-        pq.c00[e] = wq[a] * c;
-        pq.c01[e] = -wq[b] * sv;
-        pq.c10[e] = wq[a] * sv;
-        pq.c11[e] = wq[b] * c;
-        pk.c00[e] = wk[a] * c;
-        pk.c01[e] = -wk[b] * sv;
-        pk.c10[e] = wk[a] * sv;
-        pk.c11[e] = wk[b] * c;
-    }
-}
-
 template <int D, int MODE>
 __global__ void __launch_bounds__(kCtaThreads)
 qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
 {
     constexpr int LPH = D / 8;          // lanes per head
+    constexpr int NP = MODE == kRopeNone ? 1 : 4;  // pairs per lane
     const int lane = threadIdx.x & (kWarp - 1);
     const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     RowSlot s;
@@ -246,6 +194,45 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
     else
         load_batch<D, MODE>(krow, p.num_k_heads, 0, sub, li, cur);
 
+    float cs[NP], sn[NP];
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        cs[e] = 1.f;
+        sn[e] = 0.f;
+    }
+    if (MODE != kRopeNone) {
+        // Positions of this row: a row inside the sequence's T x H x W video
+        // grid (t-major, then h, then w) is 3D; every later row is 1D, counted
+        // from the end of the grid.  Without a grid every row is 1D.
+        // g: the row's index in its whole sequence (the buffer may hold one
+        // rank's slice of it, starting at row pos_offset[seq])
+        const long long g = (long long)s.local + (p.pos_offset != nullptr ? __ldg(p.pos_offset + s.seq) : 0);
+        bool is3d = false;
+        long long pt = 0, ph = 0, pw = 0;
+        long long pos1 = g;
+        if (p.rope_grid != nullptr) {
+            const long long T = __ldg(p.rope_grid + 3 * s.seq);
+            const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
+            const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
+            const long long thw = T * H * W;
+            if (g < thw) {
+                is3d = true;
+                pt = g / (H * W);
+                ph = (g / W) % H;
+                pw = g % W;
+            } else {
+                pos1 = g - thw;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            const int j = 4 * li + e;
+            const int ax = p.axis[j];
+            const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
+            const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
+            pair_cos_sin(ang, cs[e], sn[e]);
+        }
+    }
     // the weights of the lane's 8 elements, in register order
     float wq[8], wk[8];
     if (MODE == kRopeHalf) {
@@ -260,7 +247,22 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         unpack8(ld_readonly(p.k_weight + 8 * li), wk);
     }
     PairCoef pq{}, pk{};
-    row_coefficients<D, MODE>(p, s.seq, s.local, li, wq, wk, pq, pk);
+    if (MODE != kRopeNone) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int a, b;
+            pair_regs<MODE>(e, a, b);
+            const float c = cs[e % NP], sv = sn[e % NP];
+            pq.c00[e] = wq[a] * c;
+            pq.c01[e] = -wq[b] * sv;
+            pq.c10[e] = wq[a] * sv;
+            pq.c11[e] = wq[b] * c;
+            pk.c00[e] = wk[a] * c;
+            pk.c01[e] = -wk[b] * sv;
+            pk.c10[e] = wk[a] * sv;
+            pk.c11[e] = wk[b] * c;
+        }
+    }
     for (int b = 0; b < nb.n; ++b) {
         uint4 nxt[kUnroll];
         const int bn = b + 1;
@@ -278,133 +280,13 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
     }
 }
 
-// Small rows (a few KB) in large numbers: one warp takes rows_per_warp
-// consecutive valid rows, so that a warp still has enough in flight.  Its
-// work is one sequence of head batches -- a row's q batches, then its k
-// batches, then the next row's -- software-pipelined across row boundaries:
-// the next batch's loads go out before the current batch is computed, and a
-// row's angles are computed while its first batch travels.
-template <int D, int MODE>
-__global__ void __launch_bounds__(kCtaThreads)
-qk_rmsnorm_rope_rows_kernel(const __grid_constant__ QkParams p, int rows_per_warp)  // read in place: per-lane tables
-{
-    constexpr int LPH = D / 8;  // lanes per head
-    constexpr int kBatchHeads = Batches<D>::kHeads;
-    const int lane = threadIdx.x & (kWarp - 1);
-    const int wv = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-    const int total = min(max(__ldg(p.pk.cu_seqlens + p.pk.num_seqs), 0), p.pk.num_rows_padded);
-    const long long v0l = (long long)wv * rows_per_warp;
-    if (v0l >= total)
-        return;  // uniform over the warp
-    const int v0 = (int)v0l;
-    const int v1 = (int)min((long long)total, v0l + rows_per_warp);
-    const int sub = lane / LPH;  // which head of the step
-    const int li = lane % LPH;   // position inside the head: pairs 4*li .. 4*li+3
-    const Batches<D> nb(p.num_q_heads, p.num_k_heads);
-
-    // the rows are found by a cursor that runs with the loads (one batch ahead
-    // of the arithmetic); it only moves forward
-    RowCursor lc{p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded};
-    {
-        const int b = find_seq(v0, p.pk.cu_seqlens, p.pk.num_seqs, lane);
-        lc.load(b < 0 ? 0 : b);
-    }
-    int vl = v0;
-    // next valid row of the warp's range: padded row, sequence, index in it
-    auto next_row = [&](int& row, int& seq, int& local) -> bool {
-        while (vl < v1) {
-            const int r = lc.row(vl);
-            ++vl;
-            if (r >= 0) {
-                row = r;
-                seq = lc.b;
-                local = vl - 1 - lc.cs0;
-                return true;
-            }
-        }
-        return false;
-    };
-    auto load = [&](int row, int bi, uint4 (&xv)[kUnroll]) {
-        if (bi < nb.nq)
-            load_batch<D, MODE>(p.q + (int64_t)row * p.q_row_stride, p.num_q_heads, bi * kBatchHeads, sub, li, xv);
-        else
-            load_batch<D, MODE>(p.k + (int64_t)row * p.k_row_stride, p.num_k_heads, (bi - nb.nq) * kBatchHeads, sub,
-                                li, xv);
-    };
-
-    int lrow, lseq, llocal;  // the row whose batches are being loaded
-    if (!next_row(lrow, lseq, llocal))
-        return;  // uniform
-    uint4 cur[kUnroll];
-    load(lrow, 0, cur);  // travels while the weights and the row's angles are prepared
-    int lbi = 1;
-
-    // the weights of the lane's 8 elements, in register order
-    float wq[8], wk[8];
-    if (MODE == kRopeHalf) {
-        const uint2 q0 = __ldg(reinterpret_cast<const uint2*>(p.q_weight + lane_off<D, MODE>(li, 0)));
-        const uint2 q1 = __ldg(reinterpret_cast<const uint2*>(p.q_weight + lane_off<D, MODE>(li, 1)));
-        const uint2 k0 = __ldg(reinterpret_cast<const uint2*>(p.k_weight + lane_off<D, MODE>(li, 0)));
-        const uint2 k1 = __ldg(reinterpret_cast<const uint2*>(p.k_weight + lane_off<D, MODE>(li, 1)));
-        unpack8(make_uint4(q0.x, q0.y, q1.x, q1.y), wq);
-        unpack8(make_uint4(k0.x, k0.y, k1.x, k1.y), wk);
-    } else {
-        unpack8(ld_readonly(p.q_weight + 8 * li), wq);
-        unpack8(ld_readonly(p.k_weight + 8 * li), wk);
-    }
-
-    int crow = lrow;  // the row whose batches are being computed
-    PairCoef pq{}, pk{};
-    row_coefficients<D, MODE>(p, lseq, llocal, li, wq, wk, pq, pk);
-    int cbi = 0;
-    while (true) {
-        // issue the next batch: the rest of this row, else the next row's first
-        uint4 nxt[kUnroll];
-        bool more = true;
-        if (lbi < nb.n) {
-            load(lrow, lbi, nxt);
-            ++lbi;
-        } else if (next_row(lrow, lseq, llocal)) {
-            load(lrow, 0, nxt);
-            lbi = 1;
-        } else {
-            more = false;
-        }
-        if (cbi < nb.nq)
-            rms_rotate_batch<D, MODE>(p.q + (int64_t)crow * p.q_row_stride, p.num_q_heads, cbi * kBatchHeads, sub, li,
-                                      p.eps, wq, pq, cur);
-        else
-            rms_rotate_batch<D, MODE>(p.k + (int64_t)crow * p.k_row_stride, p.num_k_heads,
-                                      (cbi - nb.nq) * kBatchHeads, sub, li, p.eps, wk, pk, cur);
-        if (!more)
-            break;
-        if (++cbi == nb.n) {  // the batch just issued opens the next row
-            crow = lrow;
-            cbi = 0;
-            row_coefficients<D, MODE>(p, lseq, llocal, li, wq, wk, pq, pk);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            cur[u] = nxt[u];
-    }
-}
-
-template <int D, int MODE>
-void launch_mode(const QkParams& p, unsigned grid, int rows_per_warp, cudaStream_t stream)
-{
-    if (rows_per_warp > 1)
-        qk_rmsnorm_rope_rows_kernel<D, MODE><<<grid, kCtaThreads, 0, stream>>>(p, rows_per_warp);
-    else
-        qk_rmsnorm_rope_kernel<D, MODE><<<grid, kCtaThreads, 0, stream>>>(p);
-}
-
 template <int D>
-cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, int rows_per_warp, cudaStream_t stream)
+cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
 {
     switch (mode) {
-    case kRopeInterleaved: launch_mode<D, kRopeInterleaved>(p, grid, rows_per_warp, stream); break;
-    case kRopeHalf: launch_mode<D, kRopeHalf>(p, grid, rows_per_warp, stream); break;
-    case kRopeNone: launch_mode<D, kRopeNone>(p, grid, rows_per_warp, stream); break;
+    case kRopeInterleaved: qk_rmsnorm_rope_kernel<D, kRopeInterleaved><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeHalf: qk_rmsnorm_rope_kernel<D, kRopeHalf><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeNone: qk_rmsnorm_rope_kernel<D, kRopeNone><<<grid, kCtaThreads, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -412,27 +294,13 @@ cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, int rows_per_wa
 
 }  // namespace
 
-// Rows per warp: 1 for rows of DiT width (tens of KB); for small rows enough
-// that a warp moves about 16 KB, but only while the grid still has about 32
-// warps per SM to spread.
 cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, int rope_mode, cudaStream_t stream)
 {
-    int dev = 0, sms = 0;
-    cudaError_t e;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-    const long long row_bytes = 2LL * (p.num_q_heads + p.num_k_heads) * head_dim;
-    long long rpw = row_bytes > 0 ? 16384 / row_bytes : 1;
-    rpw = rpw < 1 ? 1 : (rpw > 8 ? 8 : rpw);
-    const long long by_rows = p.pk.num_rows_padded / (32LL * (sms > 0 ? sms : 1));
-    rpw = rpw < by_rows ? rpw : (by_rows > 1 ? by_rows : 1);
-    const long long warps = (p.pk.num_rows_padded + rpw - 1) / rpw;
-    const unsigned grid = (unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta);
+    const unsigned grid = (unsigned)((p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta);
     switch (head_dim) {
-    case 64: return launch_d<64>(p, rope_mode, grid, (int)rpw, stream);
-    case 128: return launch_d<128>(p, rope_mode, grid, (int)rpw, stream);
-    case 256: return launch_d<256>(p, rope_mode, grid, (int)rpw, stream);
+    case 64: return launch_d<64>(p, rope_mode, grid, stream);
+    case 128: return launch_d<128>(p, rope_mode, grid, stream);
+    case 256: return launch_d<256>(p, rope_mode, grid, stream);
     default: return cudaErrorInvalidValue;
     }
 }

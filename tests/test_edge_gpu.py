@@ -268,10 +268,9 @@ def test_vae_like_shapes():
 
 @pytest.mark.parametrize("mode", ["interleaved", "half"])
 @pytest.mark.parametrize("sliced", [False, True])
-def test_small_rows_several_per_warp(mode, sliced):
+def test_small_rows_many_sequences(mode, sliced):
     """Rows of 256 bytes (one q and one k head of 64) in the tens of
-    thousands: each warp takes several rows, its head batches pipelined across
-    row boundaries.  Ragged 3D grids with 1D tails, empty sequences, and (when
+    thousands, ragged 3D grids with 1D tails, empty sequences, and (when
     sliced) per-sequence position offsets, all against the oracle."""
     rng = np.random.default_rng(21 if sliced else 20)
     B = 160
@@ -281,7 +280,6 @@ def test_small_rows_several_per_warp(mode, sliced):
     grids = np.stack([rng.integers(0, 4, B), rng.integers(1, 7, B), rng.integers(1, 9, B)], axis=1)
     w = W.custom("small", lengths, padded, hidden=64, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64,
                  grids=grids, sections=(24, 20, 20), seed=9)
-    assert w.num_valid > 4 * 32 * 148          # enough rows that the launcher puts several on a warp
     po = rng.integers(0, 60, B).astype(np.int32) if sliced else None
     inp = W.qk_inputs(w)
     cs, cp, grid = P.device_packing(w)
