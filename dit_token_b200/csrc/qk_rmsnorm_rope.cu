@@ -22,10 +22,8 @@
 namespace dit {
 namespace {
 
-#ifndef DIT_QK_UNROLL
-#define DIT_QK_UNROLL 4
-#endif
-constexpr int kUnroll = DIT_QK_UNROLL;  // head vectors per lane in flight
+// Steps per head batch (head vectors per lane in one batch): 4, or 2 when
+// that fills the batches better (few heads per row).
 
 // angle mod 2*pi in fp64, then single precision: keeps the angle exact to
 // ~1e-7 rad for any position, and lets sincosf take its short path.
@@ -104,13 +102,13 @@ __device__ __forceinline__ void pair_regs(int e, int& a, int& b)
     }
 }
 
-// The heads of a row are handled in batches of kUnroll steps (HPW heads per
+// The heads of a row are handled in batches of U steps (HPW heads per
 // step): first the q heads, then the k heads.  Batch b's loads are issued
 // before batch b-1 is computed, and batch 0's before the row's angles are
 // computed, so a warp always has a batch in flight.
-template <int D>
+template <int D, int U>
 struct Batches {
-    static constexpr int kHeads = (kWarp / (D / 8)) * kUnroll;  // heads per batch
+    static constexpr int kHeads = (kWarp / (D / 8)) * U;  // heads per batch
     int nq, n;
     __device__ __forceinline__ Batches(int Hq, int Hk)
         : nq((Hq + kHeads - 1) / kHeads), n(nq + (Hk + kHeads - 1) / kHeads)
@@ -118,26 +116,26 @@ struct Batches {
     }
 };
 
-template <int D, int MODE>
-__device__ __forceinline__ void load_batch(const uint16_t* row, int H, int h0, int sub, int li, uint4 (&xv)[kUnroll])
+template <int D, int MODE, int U>
+__device__ __forceinline__ void load_batch(const uint16_t* row, int H, int h0, int sub, int li, uint4 (&xv)[U])
 {
     constexpr int HPW = kWarp / (D / 8);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
         const int h = h0 + u * HPW + sub;
         xv[u] = h < H ? load_head<D, MODE>(row + (int64_t)h * D, li) : make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
-template <int D, int MODE>
+template <int D, int MODE, int U>
 __device__ __forceinline__ void rms_rotate_batch(uint16_t* row, int H, int h0, int sub, int li, float eps,
-                                                 const float (&w)[8], const PairCoef& pc, const uint4 (&xv)[kUnroll])
+                                                 const float (&w)[8], const PairCoef& pc, const uint4 (&xv)[U])
 {
     constexpr int LPH = D / 8;
     constexpr int HPW = kWarp / LPH;
     const float inv_d = 1.0f / (float)D;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
         const int h = h0 + u * HPW + sub;
         const uint32_t wd[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
         f32x2 ss2 = f2_make(0.f, 0.f);
@@ -168,7 +166,7 @@ __device__ __forceinline__ void rms_rotate_batch(uint16_t* row, int H, int h0, i
     }
 }
 
-template <int D, int MODE>
+template <int D, int MODE, int U>
 __global__ void __launch_bounds__(kCtaThreads)
 qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
 {
@@ -184,15 +182,15 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
     const int li = lane % LPH;   // position inside the head: pairs 4*li .. 4*li+3
     uint16_t* qrow = p.q + (int64_t)s.row * p.q_row_stride;
     uint16_t* krow = p.k + (int64_t)s.row * p.k_row_stride;
-    constexpr int kBatchHeads = Batches<D>::kHeads;
-    const Batches<D> nb(p.num_q_heads, p.num_k_heads);
+    constexpr int kBatchHeads = Batches<D, U>::kHeads;
+    const Batches<D, U> nb(p.num_q_heads, p.num_k_heads);
 
     // batch 0 travels while the row's angles are computed
-    uint4 cur[kUnroll];
+    uint4 cur[U];
     if (nb.nq > 0)
-        load_batch<D, MODE>(qrow, p.num_q_heads, 0, sub, li, cur);
+        load_batch<D, MODE, U>(qrow, p.num_q_heads, 0, sub, li, cur);
     else
-        load_batch<D, MODE>(krow, p.num_k_heads, 0, sub, li, cur);
+        load_batch<D, MODE, U>(krow, p.num_k_heads, 0, sub, li, cur);
 
     float cs[NP], sn[NP];
 #pragma unroll
@@ -264,32 +262,47 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
         }
     }
     for (int b = 0; b < nb.n; ++b) {
-        uint4 nxt[kUnroll];
+        uint4 nxt[U];
         const int bn = b + 1;
         if (bn < nb.nq)
-            load_batch<D, MODE>(qrow, p.num_q_heads, bn * kBatchHeads, sub, li, nxt);
+            load_batch<D, MODE, U>(qrow, p.num_q_heads, bn * kBatchHeads, sub, li, nxt);
         else if (bn < nb.n)
-            load_batch<D, MODE>(krow, p.num_k_heads, (bn - nb.nq) * kBatchHeads, sub, li, nxt);
+            load_batch<D, MODE, U>(krow, p.num_k_heads, (bn - nb.nq) * kBatchHeads, sub, li, nxt);
         if (b < nb.nq)
-            rms_rotate_batch<D, MODE>(qrow, p.num_q_heads, b * kBatchHeads, sub, li, p.eps, wq, pq, cur);
+            rms_rotate_batch<D, MODE, U>(qrow, p.num_q_heads, b * kBatchHeads, sub, li, p.eps, wq, pq, cur);
         else
-            rms_rotate_batch<D, MODE>(krow, p.num_k_heads, (b - nb.nq) * kBatchHeads, sub, li, p.eps, wk, pk, cur);
+            rms_rotate_batch<D, MODE, U>(krow, p.num_k_heads, (b - nb.nq) * kBatchHeads, sub, li, p.eps, wk, pk, cur);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
+        for (int u = 0; u < U; ++u)
             cur[u] = nxt[u];
     }
 }
 
-template <int D>
-cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
+template <int D, int U>
+cudaError_t launch_du(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
 {
     switch (mode) {
-    case kRopeInterleaved: qk_rmsnorm_rope_kernel<D, kRopeInterleaved><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case kRopeHalf: qk_rmsnorm_rope_kernel<D, kRopeHalf><<<grid, kCtaThreads, 0, stream>>>(p); break;
-    case kRopeNone: qk_rmsnorm_rope_kernel<D, kRopeNone><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeInterleaved: qk_rmsnorm_rope_kernel<D, kRopeInterleaved, U><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeHalf: qk_rmsnorm_rope_kernel<D, kRopeHalf, U><<<grid, kCtaThreads, 0, stream>>>(p); break;
+    case kRopeNone: qk_rmsnorm_rope_kernel<D, kRopeNone, U><<<grid, kCtaThreads, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+// Batch depth: 4 steps, unless 2 fills the head batches better -- a batch of
+// 4 steps spans 4 * 32 / (D / 8) heads, and a row with, say, 8 q and 8 k heads
+// of 64 would leave half of each batch's lanes without a head.
+template <int D>
+cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
+{
+    auto batches = [&](int heads_per_batch) {
+        return (p.num_q_heads + heads_per_batch - 1) / heads_per_batch +
+               (p.num_k_heads + heads_per_batch - 1) / heads_per_batch;
+    };
+    constexpr int kHpw = kWarp / (D / 8);
+    const bool shallow = batches(2 * kHpw) * (2 * kHpw) < batches(4 * kHpw) * (4 * kHpw);
+    return shallow ? launch_du<D, 2>(p, mode, grid, stream) : launch_du<D, 4>(p, mode, grid, stream);
 }
 
 }  // namespace
