@@ -577,7 +577,8 @@ def run_dit(args):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "arith": "f32 (bf16 tensors, fp32 arithmetic, one rounding per output)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "arith": "f32 (bf16 tensors, fp32 arithmetic, one rounding per output)",
         "data": "synthetic (seeded N(0,1) activations, 1+N(0,0.02) norm weights, N(0,0.1) modulation)",
         "config": config_block(w, world),
         "step_gbs": round(step_gbs, 1), "step_hbm_frac": round(step_gbs / peak, 4),
