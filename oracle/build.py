@@ -1,6 +1,6 @@
 """Compile the CPU oracle (oracle.c) into oracle/liboracle.so.
 
-Test infrastructure only: the oracle is the plain checker that the CUDA path
+Test infrastructure only: the oracle is the plain reference that the CUDA path
 is compared against; building it does not make the product depend on it.
 """
 import os

@@ -1,4 +1,4 @@
-"""How close the kernels come to the oracle, beyond the benchmark's tolerance: on
+"""How close the kernels come to the oracle, beyond the agreement tolerance: on
 sampled rows of the video and batched varlen workloads, the share of output
 elements that are bit-identical to the oracle's result (fp64, rounded once to
 bf16) and the largest distance in bf16 units in the last place.  fp32
