@@ -17,6 +17,9 @@ pytestmark = pytest.mark.gpu
 def run_all(w, inp, stream):
     cs, cp, grid = P.device_packing(w)
     rv = W.rows_view
+    # the inputs were copied on this thread's current stream: the op stream
+    # (a non-blocking pool stream) must wait for those copies
+    stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         q, k = rv(inp["q"]), rv(inp["k"])
         dit.dit_qk_rmsnorm_rope(q, k, inp["q_weight"], inp["k_weight"], cs, cp, num_q_heads=w.num_q_heads,
