@@ -46,7 +46,7 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    tmp = LIB + ".tmp"
+    tmp = f"{LIB}.{os.getpid()}.tmp"  # per process: concurrent builds never share a file
     # Exported symbols: only the extern "C" entry points (default visibility is
     # hidden for everything else, see -fvisibility=hidden and the header).
     cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp, *sources()]

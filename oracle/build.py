@@ -20,10 +20,13 @@ def build(force: bool = False) -> str:
             return LIB
     # -O2 without -ffast-math and without -march: IEEE fp64, no contraction
     # into FMA on x86-64, so the arithmetic is exactly what the source says.
+    # a per-process temporary name: processes that build at once (several
+    # ranks) never write the same file, and the rename is atomic
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
-           "-fPIC", "-shared", "-Wall", "-Wextra", "-o", LIB + ".tmp", SRC, "-lm"]
+           "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 
