@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Throughput of the fused DiT token operators on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dit|reference]
+    python bench.py [--gpus N [--split]] [--steps K] [--warmup W] [--impl dit|reference]
                     [--workload batched_varlen] [--seed 0]
+                    [--table | --variants | --host-overhead]
 
 One step runs the whole per-token hot path once over one packed batch:
 Q/K RMSNorm + RoPE (in place), adaLN modulation, gated residual and SwiGLU,
@@ -13,13 +14,23 @@ seeded lengths in [1024, 30000] (69,829 valid tokens at seed 0), hidden 5120,
 tail.  Every op's working set (>= 1.4 GB) is larger than the 126 MB L2, so no
 flush is needed between steps.
 
-Timing: W untimed steps, then exactly K steps between CUDA events on the
-launch stream, a barrier + synchronize on both sides, the max over ranks.
+Timing: W untimed steps, then exactly K steps on the launch stream with a
+CUDA event at every step boundary (median, p10 and p90 per step in
+``step_spread``), a barrier + synchronize on both sides, the max over ranks.
 Rank 0 prints one JSON line.  ``value`` is tokens/s over all ranks; ``e2e``
 repeats the measurement through the same public API with the inputs copied
 from pinned host memory and the outputs copied back inside the timed region;
 ``roofline`` rates the dominant kernel against the measured HBM copy
-bandwidth; ``cpu_baseline`` times the plain CPU oracle on a bounded sample.
+bandwidth; ``clocks`` summarises NVML samples (every 5 ms) of the timed
+window; ``small_shapes`` times the step at the per-rank-sized shapes
+(single_stream, and long_video_slice: one rank's share of the long video
+under an 8-way row split) against the sum of the ops timed alone;
+``cpu_baseline`` times the plain CPU oracle on a bounded sample, on all host
+threads and on one.
+
+``--gpus N`` (under torch.distributed.run) gives every rank its own batch
+(weak scaling); with ``--split`` the ranks instead split ONE batch by valid
+tokens (``dit_token_b200.shard``, strong scaling), with no exchange.
 
 ``--impl reference`` times the CPU oracle alone (the only reference this
 operator set has): rank 0 runs K + W bounded samples of the same workload on
@@ -28,7 +39,8 @@ the host cores and prints the same JSON line with "impl": "reference".
 ``--table`` prints a per-op markdown table over every workload and
 ``--variants`` one over the operator variants (fp32 and per-stream
 modulation vectors, rotary layouts, grouped K heads, head_dim 256), both
-with a read-only pass over 512 MB before every timed launch (clean L2).
+with a read-only pass over 512 MB before every timed launch (clean L2);
+``--host-overhead`` prints the host time per call of every entry point.
 """
 from __future__ import annotations
 
@@ -121,14 +133,26 @@ def measured_peak():
 # ------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) of one GPU while the work runs."""
+    """SM clock, power and clock-event reasons of one GPU while the work runs.
+
+    Polls NVML every 5 ms from a background thread (query only: nothing is
+    set), so even a timed region of a few tens of milliseconds holds several
+    samples; falls back to ``nvidia-smi -lms 200`` where NVML is unavailable."""
+    # NVML clock-event reason bits that the summary names
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device: int):
-        self.samples = []
+    def __init__(self, device: int, period_s: float = 0.005):
+        self.samples = []   # (host time, sm MHz, reason names, power W)
+        self.period = period_s
         self.proc = None
+        self.stop_flag = threading.Event()
+        self.thread = None
+        self.source = None
+        self.max_mhz = None
         try:
             ident = str(torch.cuda.get_device_properties(device).uuid)
             ident = ident if ident.startswith("GPU-") else "GPU-" + ident
@@ -138,20 +162,60 @@ class ClockSampler:
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.ident.encode() if isinstance(self.ident, str) else self.ident)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.source = f"nvml every {self.period * 1e3:.0f} ms"
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        t = time.time()
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        bits = int(get_reasons(h))
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        names = [n for n, b in self.REASON_BITS.items() if bits & b]
+                        self.samples.append((t, sm, names, pw))
+                    except Exception:
+                        return
+                    self.stop_flag.wait(self.period)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.source = None
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
                  f"--id={self.ident}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi every 200 ms"
             threading.Thread(target=self._read, daemon=True).start()
         except Exception:
             self.proc = None
 
     def _read(self):
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 9:
-                self.samples.append((time.time(), parts))
+            if len(parts) != 9:
+                continue
+            try:
+                sm = float(parts[1])
+                self.max_mhz = float(parts[2])
+                pw = float(parts[3])
+            except ValueError:
+                continue
+            active = [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]
+            self.samples.append((time.time(), sm, active, pw))
 
     def stop(self):
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -160,25 +224,25 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0: float, t1: float):
-        window = [p for t, p in self.samples if t0 <= t <= t1 + 0.25]
-        rows = window or [p for _, p in self.samples]
+        """Median, min and max SM clock, reasons seen and peak power over the
+        samples taken inside [t0, t1] (all samples if none fell inside)."""
+        window = [p for p in self.samples if t0 <= p[0] <= t1]
+        rows = window or self.samples
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        def num(v):
-            try:
-                return float(v)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        reasons = set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for r in rows:
-            for name, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
-                "power_w_max": max((num(r[3]) or 0.0) for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows), "in_timed_window": bool(window)}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": self.source}
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n in r[2]})
+        return {"sm_mhz": statistics.median(sm), "sm_mhz_min": min(sm), "sm_mhz_max": max(sm),
+                "sm_max_mhz": self.max_mhz, "power_w_max": round(max(r[3] for r in rows), 1),
+                "reasons": reasons, "samples": len(rows), "in_timed_window": bool(window),
+                "window_s": round(t1 - t0, 4), "source": self.source}
+
+
+def spread(values_ms) -> dict:
+    """Median, 10th and 90th percentile of per-step (or per-launch) times, in us."""
+    v = np.asarray(list(values_ms), dtype=np.float64) * 1e3
+    return {"median_us": round(float(np.median(v)), 2), "p10_us": round(float(np.percentile(v, 10)), 2),
+            "p90_us": round(float(np.percentile(v, 90)), 2), "n": int(v.size)}
 
 
 # ------------------------------------------------------------ distributed
@@ -223,6 +287,7 @@ class Step:
         self.cs = torch.from_numpy(w.cu_seqlens).to(device)
         self.cp = torch.from_numpy(w.cu_seqlens_padded).to(device)
         self.grid = None if w.rope_grid is None else torch.from_numpy(w.rope_grid).to(device)
+        self.pos_offset = None if w.pos_offset is None else torch.from_numpy(w.pos_offsets).to(device)
         self.q, self.k = dev(host["qk"]["q"]), dev(host["qk"]["k"])
         self.wq, self.wk = dev(host["qk"]["q_weight"]), dev(host["qk"]["k_weight"])
         self.ax, self.aout = dev(host["adaln"]["x"]), dev(host["adaln"]["out"])
@@ -245,7 +310,8 @@ class Step:
         if op == "qk_rmsnorm_rope":
             d.dit_qk_rmsnorm_rope(rv(self.q), rv(self.k), self.wq, self.wk, self.cs, self.cp,
                                   num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
-                                  rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps)
+                                  rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
+                                  pos_offset=self.pos_offset)
         elif op == "adaln_modulate":
             d.dit_adaln_modulate(rv(self.ax), self.mod[:, 0], self.mod[:, 1], self.cs, self.cp,
                                  out=rv(self.aout), eps=w.eps)
@@ -312,31 +378,34 @@ def host_inputs(w: W.Workload) -> dict:
 
 def time_device(step: Step, steps: int, warmup: int, device):
     """K steps timed bare (the headline: nothing between the kernels but the
-    kernels), then K more with CUDA events around every op for the per-op
-    means (the events themselves cost a little, so they stay out of the
-    headline pass)."""
+    kernels and one CUDA event per step boundary, which gives each step's
+    time), then K more with CUDA events around every op for the per-op
+    figures (those events sit between the kernels, so they stay out of the
+    headline pass).  Returns (elapsed ms of the K headline steps, per-step ms,
+    {op: per-launch ms}, host time window of the headline pass)."""
     stream = torch.cuda.current_stream(device)
     for _ in range(warmup):
         step.run()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     barrier()
     torch.cuda.synchronize(device)
     t_host0 = time.time()
-    start.record(stream)
-    for _ in range(steps):
+    marks[0].record(stream)
+    for i in range(steps):
         step.run()
-    end.record(stream)
+        marks[i + 1].record(stream)
     torch.cuda.synchronize(device)
     t_host1 = time.time()
     barrier()
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = marks[0].elapsed_time(marks[-1])
+    step_ms = [marks[i].elapsed_time(marks[i + 1]) for i in range(steps)]
     per_op = {op: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(steps)] for op in OPS}
     for i in range(steps):
         step.run({op: per_op[op][i] for op in OPS})
     torch.cuda.synchronize(device)
-    op_ms = {op: statistics.fmean(a.elapsed_time(b) for a, b in per_op[op]) for op in OPS}
-    return elapsed_ms, op_ms, (t_host0, t_host1)
+    op_ms = {op: [a.elapsed_time(b) for a, b in per_op[op]] for op in OPS}
+    return elapsed_ms, step_ms, op_ms, (t_host0, t_host1)
 
 
 def time_graph(step: Step, steps: int, warmup: int, device) -> float:
@@ -473,7 +542,7 @@ class OracleRunner:
         o.qk_rmsnorm_rope(self.q, self.k, self.wq, self.wk, w.cu_seqlens, w.cu_seqlens_padded,
                           num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
                           rope_grid=w.rope_grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
-                          rows=rows, q_out=self.outs["q"], k_out=self.outs["k"])
+                          rows=rows, q_out=self.outs["q"], k_out=self.outs["k"], pos_offset=w.pos_offsets)
         o.adaln_modulate(self.ax, self.mod, self.mod[C:], w.cu_seqlens, w.cu_seqlens_padded, hidden=C,
                          eps=w.eps, mod_seq_stride=6 * C, rows=rows, out=self.outs["a"])
         o.gated_residual(self.rx, self.ry, self.mod[2 * C:], w.cu_seqlens, w.cu_seqlens_padded, hidden=C,
@@ -498,26 +567,234 @@ class OracleRunner:
         return int(max(16, min(self.w.num_valid, n * budget_s / max(t, 1e-6))))
 
 
-def cpu_baseline(w: W.Workload, host: dict, budget_s: float = 12.0) -> dict:
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w: W.Workload, host: dict, budget_s: float = 12.0, budget_1t_s: float = 5.0) -> dict:
+    """The oracle as it stands on a bounded seeded sample of the workload's
+    valid tokens: once with OpenMP on every host thread it gets, once with
+    one thread."""
     runner = OracleRunner(w, host)
     n = runner.calibrate(budget_s)
     rows = runner.sample(n, seed=11)
     t = runner.run(rows)
-    return {"value": rows.size / t, "unit": UNIT, "cores": runner.threads(), "kind": "oracle",
+    threads = runner.threads()
+    runner.o.set_num_threads(1)
+    try:
+        n1 = runner.calibrate(budget_1t_s)
+        rows1 = runner.sample(n1, seed=12)
+        t1 = runner.run(rows1)
+    finally:
+        runner.o.set_num_threads(threads)
+    return {"value": rows.size / t, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{rows.size} of {w.num_valid} valid tokens of {w.name} (seeded random rows), "
-                      f"all four ops per token, fp64 C oracle, {t:.1f} s"}
+                      f"all four ops per token, fp64 C oracle, {t:.1f} s on {threads} threads",
+            "value_1thread": rows1.size / t1,
+            "sample_1thread": f"{rows1.size} seeded random valid tokens, {t1:.1f} s on 1 thread",
+            "cpu_model": cpu_model(), "host_threads": os.cpu_count()}
 
 
 # ------------------------------------------------------------ main
 
-def config_block(w: W.Workload, n: int) -> dict:
-    return {"workload": w.name, "num_seqs": w.num_seqs, "valid_tokens": w.num_valid,
-            "padded_rows": w.num_rows_padded, "lengths": list(w.lengths), "hidden": w.hidden,
-            "heads": f"{w.num_q_heads}+{w.num_k_heads}x{w.head_dim}", "inner": w.inner,
-            "rope": "3d t/h/w 44/42/42 on 24x42 frames + 1d tail" if w.grids else "1d",
-            "ops_per_step": list(OPS),
-            "l2": "inputs larger than L2 (each op moves >= 1.4 GB per step vs 126 MB L2)",
-            "parallelism": f"dp{n}: every GPU runs its own batch, no collective on the data path"}
+def config_block(w: W.Workload, n: int, split: bool = False, whole: W.Workload = None) -> dict:
+    src = whole if whole is not None else w
+    cfg = {"workload": src.name, "num_seqs": src.num_seqs, "valid_tokens": src.num_valid,
+           "padded_rows": src.num_rows_padded, "lengths": list(src.lengths), "hidden": src.hidden,
+           "heads": f"{src.num_q_heads}+{src.num_k_heads}x{src.head_dim}", "inner": src.inner,
+           "rope": "3d t/h/w 44/42/42 on 24x42 frames + 1d tail" if src.grids else "1d",
+           "ops_per_step": list(OPS),
+           "l2": "inputs larger than L2 (each op moves >= 1.4 GB per step vs 126 MB L2)",
+           "parallelism": f"dp{n}: every GPU runs its own batch, no collective on the data path"}
+    if split:
+        cfg["parallelism"] = (f"rows{n}: one batch split by valid tokens over {n} ranks (contiguous, count-"
+                              "balanced slices with whole-sequence rotary positions), no collective on the "
+                              "data path")
+        cfg["rank0_slice"] = {"valid_tokens": w.num_valid, "padded_rows": w.num_rows_padded,
+                              "lengths": list(w.lengths), "pos_offset": list(w.pos_offset or ())}
+        cfg["l2"] = "per-rank slices; each op's working set per step is larger than L2 at 8 ranks or fewer"
+    return cfg
+
+
+def split_workload(w: W.Workload, rank: int, world: int) -> W.Workload:
+    """Rank ``rank``'s slice of one batch split over ``world`` ranks by valid
+    tokens (``dit_token_b200.shard``): its sequences' pieces, their padding,
+    grids and whole-sequence position offsets.  Every rank draws its slice's
+    values from the batch's seed (the timing depends on shapes, not values)."""
+    from dit_token_b200.shard import shard_packing
+    sh = shard_packing(w.cu_seqlens, w.cu_seqlens_padded, w.rope_grid, rank, world)
+    return dataclasses.replace(
+        w, name=f"{w.name} rank {rank}/{world}", lengths=tuple(int(v) for v in np.diff(sh.cu_seqlens)),
+        padded=tuple(int(v) for v in np.diff(sh.cu_seqlens_padded)),
+        grids=None if sh.rope_grid is None else tuple(tuple(int(t) for t in g) for g in sh.rope_grid),
+        pos_offset=tuple(int(v) for v in sh.pos_offset), seed=w.seed + 7919 * rank)
+
+
+def plan(args, rank: int, world: int):
+    """(this rank's workload, the whole job's workload, valid tokens per step
+    over all ranks, scaling mode)."""
+    w0 = W.scaled(W.workload(args.workload, args.seed), args.scale)
+    if getattr(args, "split", False):
+        return split_workload(w0, rank, world), w0, w0.num_valid, "strong"
+    return dataclasses.replace(w0, seed=data_seed(args.seed, rank)), w0, w0.num_valid * world, "weak"
+
+
+SMALL_SHAPES = ("single_stream", "long_video_slice")
+
+
+def time_small_shapes(device, seed: int, steps: int = 100, reps: int = 30) -> dict:
+    """The four-op step at the per-rank-sized shapes (one rank's slice of the
+    long video under an 8-way split, and the single-stream workload): per-step
+    times of back-to-back eager steps and of graph replays, against the sum of
+    each op timed alone (an L2-evicting read before every launch, median of
+    ``reps``)."""
+    flush = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)  # 512 MB, 4x L2
+    out = {}
+    for name in SMALL_SHAPES:
+        w = W.workload(name, seed)
+        step = Step(w, host_inputs(w), device)
+        stream = torch.cuda.current_stream(device)
+        for _ in range(5):
+            step.run()
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        torch.cuda.synchronize(device)
+        marks[0].record(stream)
+        for i in range(steps):
+            step.run()
+            marks[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        step_ms = [marks[i].elapsed_time(marks[i + 1]) for i in range(steps)]
+        graph_ms = time_graph(step, steps, 5, device)
+        alone = {}
+        for op in OPS:
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for a, b in ev:
+                flush.sum()  # a read-only pass: the kernel starts on clean L2 lines
+                a.record()
+                step.run_op(op)
+                b.record()
+            torch.cuda.synchronize(device)
+            alone[op] = statistics.median(a.elapsed_time(b) for a, b in ev)
+        abytes = algorithmic_bytes(w)
+        peak, _ = measured_peak()
+        med = statistics.median(step_ms)
+        out[name] = {
+            "valid_tokens": w.num_valid, "hidden": w.hidden, "inner": w.inner,
+            "step": spread(step_ms), "graph_us_per_step": round(graph_ms * 1e3, 2),
+            "tokens_per_s": round(w.num_valid / (med / 1e3), 1),
+            "step_hbm_frac": round(sum(abytes.values()) / (med / 1e3) / 1e9 / peak, 4),
+            "ops_alone_us": {op: round(v * 1e3, 2) for op, v in alone.items()},
+            "ops_alone_frac": {op: round(abytes[op] / (alone[op] / 1e3) / 1e9 / peak, 4) for op in OPS},
+            "sum_alone_us": round(sum(alone.values()) * 1e3, 2),
+            "step_over_sum_alone": round(med / sum(alone.values()), 4)}
+        del step
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure(args, w: W.Workload, device, world: int) -> dict:
+    """Every GPU measurement of the line, this rank's own numbers (ms)."""
+    host = host_inputs(w)
+    step = Step(w, host, device)
+    sampler = ClockSampler(device.index or 0)
+    sampler.start()
+    elapsed_ms, step_list, op_lists, (h0, h1) = time_device(step, args.steps, args.warmup, device)
+    sampler.stop()
+    m = {"elapsed_ms": elapsed_ms, "step_ms": step_list, "op_ms": op_lists, "clocks": sampler.summary(h0, h1)}
+    m["next_ms"] = time_next_ops(step, args.steps, args.warmup, device, args.scale)
+    m["graph_ms"] = time_graph(step, args.steps, args.warmup, device)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    # two device buffer sets let consecutive end-to-end steps overlap; the
+    # small profiling-size runs (--scale < 1) keep one to stay small
+    sets = [step, Step(w, host, device)] if args.scale >= 1.0 else [step]
+    m["e2e"] = time_e2e(sets, e2e_steps, min(args.warmup, 3), device)
+    m["e2e_steps"] = e2e_steps
+    del sets, step
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_small_shapes:
+        m["small_shapes"] = time_small_shapes(device, args.seed)
+    if world == 1 and not args.no_cpu_baseline:
+        m["cpu_baseline"] = cpu_baseline(w, host, args.cpu_budget)
+    return m
+
+
+def assemble(args, world: int, w: W.Workload, whole: W.Workload, tokens: int, scaling: str, m: dict,
+             device) -> dict:
+    """The JSON line from this rank's measurements; every rank takes the same
+    collective steps (max over ranks of each time)."""
+    max_ms = reduce_max(m["elapsed_ms"], device)
+    op_ms_max = {op: reduce_max(statistics.fmean(v), device) for op, v in m["op_ms"].items()}
+    next_ms = {k: reduce_max(v, device) for k, v in m["next_ms"].items()}
+    graph_ms = reduce_max(m["graph_ms"], device)
+    timed_e2e = m["e2e"]
+    e2e_steps = m["e2e_steps"]
+    if timed_e2e is None:
+        e2e = {"value": None, "unit": UNIT,
+               "unavailable": "the host could not pin the step's input and output buffers on every rank"}
+    else:
+        e2e_ms, h2d, d2h = timed_e2e
+        e2e_max = reduce_max(e2e_ms, device)
+        e2e = {"value": round(tokens * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": round(e2e_max / e2e_steps, 3),
+               "schedule": "per-op upload / kernel / download on 3 streams, 2 device buffer sets"}
+    value = tokens * args.steps / (max_ms / 1e3)
+    abytes = algorithmic_bytes(w)
+    peak, peak_kind = measured_peak()
+    ops = {}
+    for op in OPS:
+        gbs = abytes[op] / (op_ms_max[op] / 1e3) / 1e9
+        ops[op] = {"us": round(op_ms_max[op] * 1e3, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                   "bytes": abytes[op], "spread": spread(m["op_ms"][op])}
+    dom = max(OPS, key=lambda o: op_ms_max[o])
+    dom_gbs = abytes[dom] / (op_ms_max[dom] / 1e3) / 1e9
+    step_gbs = sum(abytes.values()) / (max_ms / args.steps / 1e3) / 1e9
+    fshape = frames_shape(args.scale)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": scaling, "vs_baseline": None, "dtype": "bf16",
+        "arith": "f32 (bf16 tensors, fp32 arithmetic, one rounding per output)",
+        "data": "synthetic (seeded N(0,1) activations, 1+N(0,0.02) norm weights, N(0,0.1) modulation)",
+        "config": config_block(w, world, split=scaling == "strong", whole=whole),
+        "step_gbs": round(step_gbs, 1), "step_hbm_frac": round(step_gbs / peak, 4),
+        "step_spread": spread(m["step_ms"]),
+        "ops": ops,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth", "unit": "GB/s",
+                     "frac": round(dom_gbs / peak, 4), "traffic": profiled_traffic(dom, w.name),
+                     "algorithmic_bytes": abytes[dom]},
+        "gpu_launches": len(OPS) * args.steps,
+        "next_ops": {
+            "gated_residual_adaln": {
+                "us": round(next_ms["gated_residual_adaln"] * 1e3, 2),
+                "gbs": round(8 * w.hidden * w.num_valid / (next_ms["gated_residual_adaln"] / 1e3) / 1e9, 1),
+                "bytes": 8 * w.hidden * w.num_valid,
+                "unfused_us": round((op_ms_max["gated_residual"] + op_ms_max["adaln_modulate"]) * 1e3, 2)},
+            "frames_to_u8": {
+                "workload": f"fp32 {list(fshape)} -> uint8 BTHWC (the pages' 10 s 1344x768 "
+                            "request: 243 frames)",
+                "us": round(next_ms["frames_to_u8"] * 1e3, 2),
+                "gbs": round(5 * math.prod(fshape) / (next_ms["frames_to_u8"] / 1e3) / 1e9, 1),
+                "bytes": 5 * math.prod(fshape)},
+        },
+        "e2e": e2e,
+        "graph": {"ms_per_step": round(graph_ms, 4), "steps": args.steps,
+                  "note": "the same step captured once in a CUDA graph and replayed; value uses the eager step"},
+        "clocks": m["clocks"],
+    }
+    if "small_shapes" in m:
+        line["small_shapes"] = m["small_shapes"]
+    if "cpu_baseline" in m:
+        line["cpu_baseline"] = m["cpu_baseline"]
+    return line
 
 
 def run_dit(args):
@@ -532,82 +809,9 @@ def run_dit(args):
     if rank == 0 or world == 1:
         build.build()
     barrier()
-    w0 = W.scaled(W.workload(args.workload, args.seed), args.scale)
-    w = dataclasses.replace(w0, seed=data_seed(args.seed, rank))
-    host = host_inputs(w)
-    step = Step(w, host, device)
-    sampler = ClockSampler(local)
-    sampler.start()
-    elapsed_ms, op_ms, (h0, h1) = time_device(step, args.steps, args.warmup, device)
-    sampler.stop()
-    clocks = sampler.summary(h0, h1)
-    max_ms = reduce_max(elapsed_ms, device)
-    op_ms_max = {op: reduce_max(v, device) for op, v in op_ms.items()}
-    next_ms = {k: reduce_max(v, device)
-               for k, v in time_next_ops(step, args.steps, args.warmup, device, args.scale).items()}
-    graph_ms = reduce_max(time_graph(step, args.steps, args.warmup, device), device)
-    e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    # two device buffer sets let consecutive end-to-end steps overlap; the
-    # small profiling-size runs (--scale < 1) keep one to stay small
-    sets = [step, Step(w, host, device)] if args.scale >= 1.0 else [step]
-    timed_e2e = time_e2e(sets, e2e_steps, min(args.warmup, 3), device)
-    if timed_e2e is None:
-        e2e = {"value": None, "unit": UNIT,
-               "unavailable": "the host could not pin the step's input and output buffers on every rank"}
-    else:
-        e2e_ms, h2d, d2h = timed_e2e
-        e2e_max = reduce_max(e2e_ms, device)
-        e2e = {"value": round(w.num_valid * world * e2e_steps / (e2e_max / 1e3), 1), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-               "ms_per_step": round(e2e_max / e2e_steps, 3),
-               "schedule": "per-op upload / kernel / download on 3 streams, 2 device buffer sets"}
-
-    tokens = w.num_valid * world
-    value = tokens * args.steps / (max_ms / 1e3)
-    abytes = algorithmic_bytes(w)
-    peak, peak_kind = measured_peak()
-    ops = {}
-    for op in OPS:
-        gbs = abytes[op] / (op_ms_max[op] / 1e3) / 1e9
-        ops[op] = {"us": round(op_ms_max[op] * 1e3, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
-                   "bytes": abytes[op]}
-    dom = max(OPS, key=lambda o: op_ms_max[o])
-    dom_gbs = abytes[dom] / (op_ms_max[dom] / 1e3) / 1e9
-    step_gbs = sum(abytes.values()) / (max_ms / args.steps / 1e3) / 1e9
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "arith": "f32 (bf16 tensors, fp32 arithmetic, one rounding per output)",
-        "data": "synthetic (seeded N(0,1) activations, 1+N(0,0.02) norm weights, N(0,0.1) modulation)",
-        "config": config_block(w, world),
-        "step_gbs": round(step_gbs, 1), "step_hbm_frac": round(step_gbs / peak, 4),
-        "ops": ops,
-        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak,
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth", "unit": "GB/s",
-                     "frac": round(dom_gbs / peak, 4), "traffic": profiled_traffic(dom, w.name),
-                     "algorithmic_bytes": abytes[dom]},
-        "gpu_launches": len(OPS) * args.steps,
-        "next_ops": {
-            "gated_residual_adaln": {
-                "us": round(next_ms["gated_residual_adaln"] * 1e3, 2),
-                "gbs": round(8 * w.hidden * w.num_valid / (next_ms["gated_residual_adaln"] / 1e3) / 1e9, 1),
-                "bytes": 8 * w.hidden * w.num_valid,
-                "unfused_us": round((op_ms_max["gated_residual"] + op_ms_max["adaln_modulate"]) * 1e3, 2)},
-            "frames_to_u8": {
-                "workload": f"fp32 {list(frames_shape(args.scale))} -> uint8 BTHWC (the pages' 10 s 1344x768 "
-                            "request: 243 frames)",
-                "us": round(next_ms["frames_to_u8"] * 1e3, 2),
-                "gbs": round(5 * math.prod(frames_shape(args.scale)) / (next_ms["frames_to_u8"] / 1e3) / 1e9, 1),
-                "bytes": 5 * math.prod(frames_shape(args.scale))},
-        },
-        "e2e": e2e,
-        "graph": {"ms_per_step": round(graph_ms, 4), "steps": args.steps,
-                  "note": "the same step captured once in a CUDA graph and replayed; value uses the eager step"},
-        "clocks": clocks,
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, host, args.cpu_budget)
+    w, whole, tokens, scaling = plan(args, rank, world)
+    m = measure(args, w, device, world)
+    line = assemble(args, world, w, whole, tokens, scaling, m, device)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -799,6 +1003,94 @@ def run_variants(args):
     torch.cuda.empty_cache()
 
 
+def run_host_overhead(args):
+    """Host time per call of every entry point on the tiny workload: 1,000
+    calls back to back with no synchronization (the GPU queue absorbs them),
+    once through the Python binding and once as a bare C-ABI call through
+    ctypes with its arguments prepared beforehand (what a C caller pays, plus
+    ctypes' own few hundred ns).  Markdown on stdout."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from dit_token_b200 import build
+    build.build()
+    import ctypes
+    import dit_token_b200 as dit
+    L = dit.library()
+    w = W.workload("tiny", args.seed)
+    step = Step(w, host_inputs(w), device)
+    rv = W.rows_view
+    C, I = w.hidden, w.inner
+    st = torch.cuda.current_stream(device).cuda_stream
+    cs, cp = step.cs.data_ptr(), step.cp.data_ptr()
+    B, R = w.num_seqs, w.num_rows_padded
+    q, k, ax, ao = rv(step.q), rv(step.k), rv(step.ax), rv(step.aout)
+    rx, ry, ro = rv(step.rx), rv(step.ry), rv(step.rout)
+    ab, so = rv(step.ab), rv(step.sout)
+    m = step.mod
+    norm = torch.empty_like(ro)
+    flag = torch.empty(2, dtype=torch.int32, device=device)
+    cs2 = torch.empty(2 * B + 1, dtype=torch.int32, device=device)
+    cp2 = torch.empty_like(cs2)
+    grid1 = torch.tensor([[1, 10, 20]], dtype=torch.int32, device=device)
+    frames = W.frames_input((1, 3, 2, 16, 32)).to(device)
+    fout = torch.empty((1, 2, 16, 32, 3), dtype=torch.uint8, device=device)
+    qs, ks = q.stride(0), k.stride(0)
+    hd = w.head_dim
+    raw = {
+        "dit_qk_rmsnorm_rope": (L.dit_qk_rmsnorm_rope, (
+            q.data_ptr(), qs, k.data_ptr(), ks, step.wq.data_ptr(), step.wk.data_ptr(), cs, cp, B, R,
+            w.num_q_heads, w.num_k_heads, hd, None, 0, 0, 0, 10000.0, 1e-6, st)),
+        "dit_adaln_modulate": (L.dit_adaln_modulate, (
+            ax.data_ptr(), C, ao.data_ptr(), C, m[:, 0].data_ptr(), m[:, 1].data_ptr(), 6 * C, cs, cp, B, R, C,
+            1e-6, st)),
+        "dit_gated_residual": (L.dit_gated_residual, (
+            rx.data_ptr(), C, ry.data_ptr(), C, m[:, 2].data_ptr(), 6 * C, ro.data_ptr(), C, cs, cp, B, R, C, st)),
+        "dit_swiglu": (L.dit_swiglu, (
+            ab.data_ptr(), 2 * I, ab[:, I:].data_ptr(), 2 * I, so.data_ptr(), I, cs, cp, B, R, I, st)),
+        "dit_gated_residual_adaln": (L.dit_gated_residual_adaln, (
+            rx.data_ptr(), C, ry.data_ptr(), C, m[:, 2].data_ptr(), 6 * C, m[:, 3].data_ptr(), m[:, 4].data_ptr(),
+            6 * C, ro.data_ptr(), C, norm.data_ptr(), C, cs, cp, B, R, C, 1e-6, st)),
+        "dit_validate_seqlens": (L.dit_validate_seqlens, (cs, cp, B, R, flag.data_ptr(), st)),
+        "dit_av_stream_seqlens": (L.dit_av_stream_seqlens, (
+            cs, cp, grid1.data_ptr(), None, B, cs2.data_ptr(), cp2.data_ptr(), st)),
+        "dit_frames_to_u8": (L.dit_frames_to_u8, (
+            ctypes.c_void_p(frames.data_ptr()), 1, 3, 2, 16, 32, 0, ctypes.c_void_p(fout.data_ptr()), st)),
+    }
+    binding = {
+        "dit_qk_rmsnorm_rope": lambda: step.run_op("qk_rmsnorm_rope"),
+        "dit_adaln_modulate": lambda: step.run_op("adaln_modulate"),
+        "dit_gated_residual": lambda: step.run_op("gated_residual"),
+        "dit_swiglu": lambda: step.run_op("swiglu"),
+        "dit_gated_residual_adaln": lambda: dit.dit_gated_residual_adaln(
+            rx, ry, m[:, 2], m[:, 3], m[:, 4], step.cs, step.cp, res_out=ro, norm_out=norm, eps=w.eps),
+        "dit_validate_seqlens": lambda: dit.dit_validate_seqlens(step.cs, step.cp, R, flag=flag),
+        "dit_av_stream_seqlens": lambda: dit.dit_av_stream_seqlens(step.cs, step.cp, grid1, out=(cs2, cp2)),
+        "dit_frames_to_u8": lambda: dit.dit_frames_to_u8(frames, layout="bthwc", out=fout),
+    }
+    n = 1000
+    print("| entry point | host us per call, C ABI via ctypes | host us per call, Python binding |")
+    print("|---|---|---|")
+    for name, (fn, a) in raw.items():
+        for _ in range(20):
+            assert fn(*a) == 0, name
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        for _ in range(n):
+            fn(*a)
+        t1 = time.perf_counter()
+        torch.cuda.synchronize(device)
+        bfn = binding[name]
+        for _ in range(20):
+            bfn()
+        torch.cuda.synchronize(device)
+        t2 = time.perf_counter()
+        for _ in range(n):
+            bfn()
+        t3 = time.perf_counter()
+        torch.cuda.synchronize(device)
+        print(f"| {name} | {(t1 - t0) / n * 1e6:.2f} | {(t3 - t2) / n * 1e6:.2f} |", flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -813,10 +1105,17 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-shapes", action="store_true",
+                    help="skip the step timing at the per-rank-sized shapes (single_stream, long_video_slice)")
+    ap.add_argument("--split", action="store_true",
+                    help="with --gpus N: the ranks split ONE batch by rows (strong scaling) instead of each "
+                         "running its own batch (weak scaling, the default)")
     ap.add_argument("--table", action="store_true",
                     help="print a per-op markdown table over every workload instead of the JSON line")
     ap.add_argument("--variants", action="store_true",
                     help="print a markdown table of the operator variants instead of the JSON line")
+    ap.add_argument("--host-overhead", action="store_true",
+                    help="print the host time per call of every entry point (tiny workload, no sync)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -824,7 +1123,9 @@ def main(argv=None):
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
-    if args.table:
+    if args.host_overhead:
+        run_host_overhead(args)
+    elif args.table:
         run_table(args)
     elif args.variants:
         run_variants(args)

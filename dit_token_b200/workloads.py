@@ -19,7 +19,16 @@ single_stream      1     8192                    8320     2048    16x128  5632
 video              1     16x24x42 + 128 audio    16384    3072    24x128  8192
 long_video         1     61x24x42 + 400 audio    61952    3072    24x128  8192
 batched_varlen     4     U[1024, 30000] each     x128     5120    40x128  13824
+long_video_slice   1     7336 video + 400 audio  7800     3072    24x128  8192
 =================  ====  ======================  =======  ======  ======  =====
+
+``long_video_slice`` is the share one rank holds when long_video's rows are
+split over 8 ranks (the serving configuration runs 8-way sequence
+parallelism, "MiniMax H3 通过 vLLM-Omni 实现 FastH3 实时推理", "FastH3
+推理配置"): rank 7 of 8 in ``shard.shard_packing``, i.e. whole-sequence rows
+54152 .. 61887 (the last 7336 video rows, the 400 audio rows) and the 64
+padding rows, with ``pos_offset`` = 54152 so its rows keep their
+whole-sequence rotary positions.
 
 Value distributions: activations N(0, 1); RMSNorm weights 1 + N(0, 0.02);
 modulation vectors (shift, scale, gate) N(0, 0.1).  Draws are fp32 normals
@@ -48,7 +57,10 @@ _CHUNK = 1 << 22
 _SLOT = {"q": 0, "k": 1, "q_weight": 2, "k_weight": 3, "adaln_x": 4, "mod": 5,
          "res_x": 6, "res_y": 7, "ab": 8, "mod_av": 9}
 
-WORKLOAD_NAMES = ("tiny", "single_stream", "video", "long_video", "batched_varlen")
+WORKLOAD_NAMES = ("tiny", "single_stream", "video", "long_video", "batched_varlen", "long_video_slice")
+
+# The rank whose share of long_video is long_video_slice, and the rank count.
+SLICE_RANK, SLICE_WORLD = 7, 8
 
 # Video latent frame of the video-shaped workloads: H x W = 24 x 42.
 _FRAME_H, _FRAME_W = 24, 42
@@ -70,6 +82,9 @@ class Workload:
     rope_theta: float = 10000.0
     eps: float = 1e-6
     seed: int = 0
+    # whole-sequence index of each sequence's first row (one rank's slice of
+    # longer sequences), or None: every sequence starts at its row 0
+    pos_offset: Optional[Tuple[int, ...]] = None
 
     @property
     def num_seqs(self) -> int:
@@ -96,6 +111,10 @@ class Workload:
         if self.grids is None:
             return None
         return np.asarray(self.grids, dtype=np.int32).reshape(-1, 3)
+
+    @property
+    def pos_offsets(self) -> Optional[np.ndarray]:
+        return None if self.pos_offset is None else np.asarray(self.pos_offset, dtype=np.int32)
 
     @property
     def qk_width(self) -> Tuple[int, int]:
@@ -137,6 +156,15 @@ def workload(name: str, seed: int = 0) -> Workload:
         grids = tuple((L // (_FRAME_H * _FRAME_W), _FRAME_H, _FRAME_W) for L in lengths)
         return Workload(name, lengths, padded, 5120, 40, 40, 128, 13824,
                         grids=grids, sections=(44, 42, 42), seed=seed)
+    if name == "long_video_slice":
+        from .shard import shard_packing
+        full = workload("long_video", seed)
+        sh = shard_packing(full.cu_seqlens, full.cu_seqlens_padded, full.rope_grid, SLICE_RANK, SLICE_WORLD)
+        return Workload(name, tuple(int(v) for v in np.diff(sh.cu_seqlens)),
+                        tuple(int(v) for v in np.diff(sh.cu_seqlens_padded)), full.hidden, full.num_q_heads,
+                        full.num_k_heads, full.head_dim, full.inner,
+                        grids=tuple(tuple(int(t) for t in g) for g in sh.rope_grid), sections=full.sections,
+                        seed=seed, pos_offset=tuple(int(v) for v in sh.pos_offset))
     raise KeyError(f"unknown workload {name!r}; known: {WORKLOAD_NAMES}")
 
 
@@ -158,6 +186,8 @@ def scaled(w: Workload, factor: float) -> Workload:
         else:  # keep the audio tail, shrink the frames
             grids = tuple((max(0, (L - (L0 - T * H * Wd)) // frame), _FRAME_H, _FRAME_W)
                           for L, L0, (T, H, Wd) in zip(lengths, w.lengths, w.grids))
+    if w.pos_offset is not None:
+        raise ValueError(f"{w.name} is a slice of longer sequences and cannot be scaled")
     return Workload(f"{w.name}@{factor:g}", lengths, padded, w.hidden, w.num_q_heads, w.num_k_heads,
                     w.head_dim, w.inner, grids, w.sections, w.rope_theta, w.eps, w.seed)
 
@@ -307,7 +337,9 @@ def frames_input(shape=FRAMES_SHAPE, seed: int = 0) -> torch.Tensor:
 
 def sample_rows(w: Workload, per_seq: int, seed: int = 1234) -> np.ndarray:
     """Padded indices of a seeded sample of valid rows: each sequence's first
-    and last valid row plus up to ``per_seq`` others."""
+    and last valid row, for a sequence with a T x H x W grid the rows at the
+    grid's edges (local W - 1, H*W - 1, T*H*W - 1 -- the largest 3D position --
+    and T*H*W, the first row after the grid), plus up to ``per_seq`` others."""
     rng = np.random.default_rng(seed)
     cp = w.cu_seqlens_padded
     picks = []
@@ -315,6 +347,10 @@ def sample_rows(w: Workload, per_seq: int, seed: int = 1234) -> np.ndarray:
         if L == 0:
             continue
         local = {0, L - 1}
+        if w.grids is not None:
+            T, H, Wd = w.grids[b]
+            off = 0 if w.pos_offset is None else w.pos_offset[b]
+            local.update(r - off for r in (Wd - 1, H * Wd - 1, T * H * Wd - 1, T * H * Wd) if 0 <= r - off < L)
         local.update(int(v) for v in rng.choice(L, size=min(per_seq, L), replace=False))
         picks.extend(cp[b] + np.array(sorted(local), dtype=np.int64))
     return np.asarray(picks, dtype=np.int64)

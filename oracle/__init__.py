@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
                      "oracle_qk_rmsnorm_rope_shard",
                      "oracle_num_threads"):
             getattr(L, name).restype = ctypes.c_int
+        L.oracle_set_num_threads.argtypes = [i32]
+        L.oracle_set_num_threads.restype = None
         _lib = L
     return _lib
 
@@ -160,6 +162,11 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
 
 def num_threads() -> int:
     return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads for the following oracle calls (results do not depend on it)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def qk_rmsnorm_rope(q, k, q_weight, k_weight, cu_seqlens, cu_seqlens_padded, *,

@@ -647,3 +647,15 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Thread count for the following calls (harness control for timing the
+ * oracle on one core; the arithmetic does not depend on it). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -233,6 +233,7 @@ int oracle_frames_to_u8(const float* x, int64_t batch, int64_t channels, int64_t
 
 /* Number of OpenMP threads the oracle's row loops use (1 without OpenMP). */
 int oracle_num_threads(void);
+void oracle_set_num_threads(int n);
 
 #ifdef __cplusplus
 }

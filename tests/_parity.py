@@ -12,20 +12,40 @@ from _util import f64, tbits
 ABS_TOL, REL_TOL = 2e-2, 1e-2
 
 
-def assert_close(gpu_bits, ref_bits, what=""):
+def _values(b: np.ndarray) -> torch.Tensor:
+    """bf16 bit patterns (uint16) -> exact fp64 values, as a CPU tensor."""
+    t = torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(torch.int32) << 16
+    return t.view(torch.float32).to(torch.float64)
+
+
+def assert_close(gpu_bits, ref_bits, what="", chunk=1 << 26):
     """|gpu - ref| <= max(2e-2, 1e-2 |ref|) elementwise, ref = the oracle's
-    fp64 result rounded once to bf16; both must be finite."""
-    g, r = f64(gpu_bits), f64(ref_bits)
-    assert g.shape == r.shape
-    assert np.all(np.isfinite(r)), f"{what}: oracle produced non-finite values"
-    assert np.all(np.isfinite(g)), f"{what}: GPU produced non-finite values at {np.argwhere(~np.isfinite(g))[:5]}"
-    tol = np.maximum(ABS_TOL, REL_TOL * np.abs(r))
-    bad = np.abs(g - r) > tol
-    if bad.any():
-        idx = np.argwhere(bad)[:5]
-        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance, e.g. "
-                             + ", ".join(f"{tuple(i)}: gpu {g[tuple(i)]} ref {r[tuple(i)]}" for i in idx))
-    return float(np.max(np.abs(g - r))) if g.size else 0.0
+    fp64 result rounded once to bf16; both must be finite.  Works through the
+    arrays in chunks (multi-threaded torch CPU arithmetic), so whole
+    full-size outputs can be compared.  Returns the largest |gpu - ref|."""
+    g_all = np.asarray(gpu_bits, dtype=np.uint16).reshape(-1)
+    r_all = np.asarray(ref_bits, dtype=np.uint16).reshape(-1)
+    assert np.shape(gpu_bits) == np.shape(ref_bits), f"{what}: shapes differ"
+    worst = 0.0
+    for lo in range(0, g_all.size, chunk):
+        g, r = _values(g_all[lo:lo + chunk]), _values(r_all[lo:lo + chunk])
+        assert bool(torch.isfinite(r).all()), f"{what}: oracle produced non-finite values"
+        if not bool(torch.isfinite(g).all()):
+            idx = torch.nonzero(~torch.isfinite(g))[:5].flatten() + lo
+            raise AssertionError(f"{what}: GPU produced non-finite values at flat indices {idx.tolist()}")
+        err = (g - r).abs()
+        tol = torch.clamp(REL_TOL * r.abs(), min=ABS_TOL)
+        bad = err > tol
+        if bool(bad.any()):
+            idx = torch.nonzero(bad)[:5].flatten()
+            shape = np.shape(gpu_bits)
+            raise AssertionError(
+                f"{what}: {int(bad.sum())} elements of chunk {lo // chunk} out of tolerance, e.g. "
+                + ", ".join(f"{np.unravel_index(int(i) + lo, shape)}: gpu {float(g[i])} ref {float(r[i])}"
+                            for i in idx))
+        if err.numel():
+            worst = max(worst, float(err.max()))
+    return worst
 
 
 def untouched_rows(w: W.Workload) -> np.ndarray:
@@ -57,10 +77,11 @@ def gpu_qk(w, inp, rope_mode="interleaved"):
     cs, cp, grid = device_packing(w)
     q = inp["q"].cuda()
     k = inp["k"].cuda()
+    po = None if w.pos_offset is None else torch.from_numpy(w.pos_offsets).cuda()
     dit.dit_qk_rmsnorm_rope(W.rows_view(q), W.rows_view(k), inp["q_weight"].cuda(), inp["k_weight"].cuda(),
                             cs, cp, num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads,
                             head_dim=w.head_dim, rope_grid=grid, sections=w.sections,
-                            rope_theta=w.rope_theta, eps=w.eps, rope_mode=rope_mode)
+                            rope_theta=w.rope_theta, eps=w.eps, rope_mode=rope_mode, pos_offset=po)
     return q, k
 
 
@@ -114,7 +135,7 @@ def oracle_qk(w, inp, rows, rope_mode="interleaved"):
                                   w.cu_seqlens_padded, num_q_heads=w.num_q_heads,
                                   num_k_heads=w.num_k_heads, head_dim=w.head_dim, rope_grid=w.rope_grid,
                                   sections=w.sections, rope_theta=w.rope_theta, eps=w.eps, rows=rows,
-                                  rope_mode=rope_mode)
+                                  rope_mode=rope_mode, pos_offset=w.pos_offsets)
 
 
 def mod_flat(mod: torch.Tensor) -> np.ndarray:

@@ -111,3 +111,54 @@ def test_two_ranks_split_one_batch_with_global_positions():
     port = _free_port()
     mp.spawn(_shard_worker, args=(2, port, out), nprocs=2, join=True)
     assert out["rows"] and out["equal"]
+
+
+def _split_worker(rank, world, port, out):
+    """The benchmark's --split leg on CPU: each rank plans its slice of one
+    batch, its (fake) device times go through the same max-over-ranks and
+    line assembly as on the GPU."""
+    import argparse
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        lines = {}
+        for split in (True, False):
+            args = argparse.Namespace(workload="batched_varlen", seed=0, scale=1.0, split=split, steps=5,
+                                      warmup=3, e2e_steps=2)
+            w, whole, tokens, scaling = bench.plan(args, rank, world)
+            slow = 1.0 + rank                      # rank 1 is the slow one
+            m = {"elapsed_ms": 10.0 * slow, "step_ms": [2.0 * slow] * 5,
+                 "op_ms": {op: [0.5 * slow] * 5 for op in bench.OPS}, "clocks": {"sm_mhz": None},
+                 "next_ms": {"gated_residual_adaln": 0.4, "frames_to_u8": 0.6}, "graph_ms": 1.9 * slow,
+                 "e2e": (300.0 * slow, 1000, 500), "e2e_steps": 2}
+            line = bench.assemble(args, world, w, whole, tokens, scaling, m, torch.device("cpu"))
+            lines[split] = (line, w.num_valid, w.num_rows_padded, list(w.pos_offset or ()), whole.num_valid)
+        out[rank] = lines
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_leg_json_contract():
+    mgr = mp.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    mp.spawn(_split_worker, args=(2, port, out), nprocs=2, join=True)
+    (l0, n0, r0, po0, total), (l1, n1, r1, po1, _) = out[0][True], out[1][True]
+    assert n0 + n1 == total == 69829            # the slices partition the batch's valid tokens
+    assert r0 + r1 == 70144                     # ... and its padded rows
+    assert po0 == [0, 0] and po1 == [n0 - 25672, 0, 0]   # rank 1 starts inside sequence 1
+    for line in (l0, l1):
+        assert line["scaling"] == "strong" and line["n_gpus"] == 2 and line["steps"] == 5
+        assert line["config"]["parallelism"].startswith("rows2")
+        assert line["config"]["valid_tokens"] == total
+        # whole-batch tokens over the slowest rank's time
+        assert abs(line["value"] - total * 5 / 0.020) < 1.0
+        assert abs(line["e2e"]["value"] - total * 2 / 0.600) < 1.0
+        assert line["gpu_launches"] == 4 * 5
+    weak0, weak1 = out[0][False][0], out[1][False][0]
+    assert weak0["scaling"] == "weak" and weak0["config"]["parallelism"].startswith("dp2")
+    assert abs(weak0["value"] - 2 * total * 5 / 0.020) < 1.0 and weak0["value"] == weak1["value"]

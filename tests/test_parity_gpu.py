@@ -1,11 +1,10 @@
 """GPU parity of the four operators against the CPU oracle on the five seeded
 workloads, at full size and in the launch configuration the benchmark times.
 
-tiny: every valid row is compared.  Larger workloads: the first and last
-valid row of every sequence plus 64 seeded random rows per sequence are
-compared element by element (the oracle computes those rows one by one);
-every padding row and the canary rows around each buffer are checked
-bit-exactly at full size, and a second run must be bitwise identical.
+Every valid row of every workload is compared element by element with the
+oracle (which computes the whole batch), every padding row and the canary
+rows around each buffer are checked bit-exactly at full size, and a second
+run must be bitwise identical.
 """
 import pytest
 import torch
@@ -23,7 +22,7 @@ def case(request):
     w = W.workload(request.param)
     inputs = {"qk": W.qk_inputs(w), "adaln": W.adaln_inputs(w), "residual": W.residual_inputs(w),
               "swiglu": W.swiglu_inputs(w)}
-    rows = w.valid_rows() if w.name == "tiny" else W.sample_rows(w, per_seq=64)
+    rows = w.valid_rows()
     yield w, inputs, rows
     del inputs
     torch.cuda.empty_cache()
