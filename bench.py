@@ -294,6 +294,13 @@ class Step:
         self.mod = dev(host["adaln"]["mod"])
         self.rx, self.ry, self.rout = dev(host["res"]["x"]), dev(host["res"]["y"]), dev(host["res"]["out"])
         self.ab, self.sout = dev(host["swiglu"]["ab"]), dev(host["swiglu"]["out"])
+        # the views each call takes, made once (as a caller holding its
+        # activations would), so the per-call host work is the binding's own
+        rv = W.rows_view
+        self.v = {"q": rv(self.q), "k": rv(self.k), "ax": rv(self.ax), "aout": rv(self.aout),
+                  "rx": rv(self.rx), "ry": rv(self.ry), "rout": rv(self.rout), "sout": rv(self.sout),
+                  "a": rv(self.ab)[:, : w.inner], "b": rv(self.ab)[:, w.inner:],
+                  "shift": self.mod[:, 0], "scale": self.mod[:, 1], "gate": self.mod[:, 2]}
 
     def op_inputs(self, op):
         """Device tensors an op reads (what a host-resident caller must upload)."""
@@ -306,20 +313,18 @@ class Step:
                 "gated_residual": [self.rout], "swiglu": [self.sout]}[op]
 
     def run_op(self, op):
-        w, d, rv = self.w, self.dit, W.rows_view
+        w, d, v = self.w, self.dit, self.v
         if op == "qk_rmsnorm_rope":
-            d.dit_qk_rmsnorm_rope(rv(self.q), rv(self.k), self.wq, self.wk, self.cs, self.cp,
+            d.dit_qk_rmsnorm_rope(v["q"], v["k"], self.wq, self.wk, self.cs, self.cp,
                                   num_q_heads=w.num_q_heads, num_k_heads=w.num_k_heads, head_dim=w.head_dim,
                                   rope_grid=self.grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
                                   pos_offset=self.pos_offset)
         elif op == "adaln_modulate":
-            d.dit_adaln_modulate(rv(self.ax), self.mod[:, 0], self.mod[:, 1], self.cs, self.cp,
-                                 out=rv(self.aout), eps=w.eps)
+            d.dit_adaln_modulate(v["ax"], v["shift"], v["scale"], self.cs, self.cp, out=v["aout"], eps=w.eps)
         elif op == "gated_residual":
-            d.dit_gated_residual(rv(self.rx), rv(self.ry), self.mod[:, 2], self.cs, self.cp, out=rv(self.rout))
+            d.dit_gated_residual(v["rx"], v["ry"], v["gate"], self.cs, self.cp, out=v["rout"])
         else:
-            ab = rv(self.ab)
-            d.dit_swiglu(ab[:, : w.inner], ab[:, w.inner:], self.cs, self.cp, out=rv(self.sout))
+            d.dit_swiglu(v["a"], v["b"], self.cs, self.cp, out=v["sout"])
 
     def run(self, events=None):
         for op in OPS:

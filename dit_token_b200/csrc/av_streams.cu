@@ -23,6 +23,7 @@ av_stream_seqlens_kernel(const int32_t* __restrict__ cs, const int32_t* __restri
                          const int32_t* __restrict__ grid, const int32_t* __restrict__ pos_offset, int B,
                          int32_t* __restrict__ out_cs, int32_t* __restrict__ out_cp)
 {
+    grid_dependency_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i == 0) {
         out_cs[0] = cs[0];
@@ -55,9 +56,8 @@ cudaError_t launch_av_stream_seqlens(const int32_t* cu_seqlens, const int32_t* c
 {
     const int blocks = num_seqs / kCtaThreads + 1;
     const unsigned grid = (unsigned)(blocks < 1024 ? blocks : 1024);
-    av_stream_seqlens_kernel<<<grid, kCtaThreads, 0, stream>>>(cu_seqlens, cu_seqlens_padded, rope_grid, pos_offset,
-                                                               num_seqs, out_cu_seqlens, out_cu_seqlens_padded);
-    return cudaGetLastError();
+    return launch_kernel(av_stream_seqlens_kernel, grid, kCtaThreads, 0, stream, cu_seqlens, cu_seqlens_padded,
+                         rope_grid, pos_offset, (int)num_seqs, out_cu_seqlens, out_cu_seqlens_padded);
 }
 
 }  // namespace dit

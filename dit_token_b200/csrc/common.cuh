@@ -11,6 +11,18 @@ constexpr int kWarp = 32;
 constexpr int kCtaThreads = 256;          // 8 warps
 constexpr int kWarpsPerCta = kCtaThreads / kWarp;
 
+// ---------------------------------------------- dependent launches
+// Called first in every kernel, before any global-memory access: waits until
+// the kernel this one depends on (the previous one on the stream, when the
+// launch carries the programmatic-serialization attribute) has completed and
+// its writes are visible, then lets this kernel's own dependents be
+// scheduled.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ packed rows
 //
 // The packed batch holds num_seqs sequences; sequence b owns padded rows
@@ -124,6 +136,49 @@ __device__ __forceinline__ void st_stream(uint16_t* p, uint4 v)
     __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
+// NW 32-bit words (NW = 4: 16 bytes, NW = 8: 32 bytes) of a streamed row,
+// evict-first.  The 32-byte form (one 256-bit access per lane, sm_100) halves
+// the load and store instructions of a row; it needs a 32-byte aligned
+// address.
+template <int NW>
+__device__ __forceinline__ void ld_stream_words(const uint16_t* p, uint32_t (&w)[NW])
+{
+    static_assert(NW == 2 || NW == 4 || NW == 8, "8-, 16- or 32-byte accesses");
+    if constexpr (NW == 2) {
+        const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+        w[0] = v.x;
+        w[1] = v.y;
+    } else if constexpr (NW == 4) {
+        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p));
+        w[0] = v.x;
+        w[1] = v.y;
+        w[2] = v.z;
+        w[3] = v.w;
+    } else {
+        // volatile: kept in program order with the other volatile asm, so
+        // never above the grid-dependency wait
+        asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+            : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+            : "l"(p));
+    }
+}
+
+// The 32-byte store is inline assembly whose memory effect the compiler does
+// not see: use it only for output the kernel never reads back.
+template <int NW>
+__device__ __forceinline__ void st_stream_words(uint16_t* p, const uint32_t (&w)[NW])
+{
+    static_assert(NW == 2 || NW == 4 || NW == 8, "8-, 16- or 32-byte accesses");
+    if constexpr (NW == 2) {
+        __stcs(reinterpret_cast<uint2*>(p), make_uint2(w[0], w[1]));
+    } else if constexpr (NW == 4) {
+        __stcs(reinterpret_cast<uint4*>(p), make_uint4(w[0], w[1], w[2], w[3]));
+    } else {
+        asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                     "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]));
+    }
+}
+
 // 8 elements of a small vector that many rows share (norm weights, gates,
 // shifts, scales): read-only path, kept in L1/L2.
 __device__ __forceinline__ uint4 ld_readonly(const uint16_t* p)
@@ -222,6 +277,26 @@ template <bool F32>
 __device__ __forceinline__ void vec8_pairs(const void* base, int64_t elem, f32x2 (&v)[4])
 {
     vec8_unpack<F32>(vec8_load<F32>(base, elem), v);
+}
+
+// NP consecutive pairs (2 * NP elements, NP = 2 or 4) of a per-sequence
+// vector starting at element `elem`, as fp32 pairs: one 8- or 16-byte load
+// (bf16) or one or two 16-byte loads (fp32) through the read-only path.
+template <bool F32, int NP>
+__device__ __forceinline__ void vec_pairs(const void* base, int64_t elem, f32x2 (&v)[NP])
+{
+    static_assert(NP == 2 || NP == 4, "4 or 8 elements");
+    if constexpr (NP == 4) {
+        vec8_pairs<F32>(base, elem, v);
+    } else if constexpr (F32) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem));
+        v[0] = make_float2(a.x, a.y);
+        v[1] = make_float2(a.z, a.w);
+    } else {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + elem));
+        v[0] = f2_from_bf16x2(u.x);
+        v[1] = f2_from_bf16x2(u.y);
+    }
 }
 
 // fp32 pair -> bf16x2 word, round to nearest even.

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(kCtaThreads)
 frames_vec_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t T, int64_t H, int64_t W,
                   int64_t items)
 {
+    grid_dependency_wait();
     const int64_t groups = W / 16;
     for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
          it += (int64_t)gridDim.x * blockDim.x) {
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kCtaThreads)
 frames_scalar_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t C, int64_t T, int64_t H,
                      int64_t W, int32_t layout, int64_t items)
 {
+    grid_dependency_wait();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items;
          i += (int64_t)gridDim.x * blockDim.x) {
         // i enumerates the output in its own order, so stores are coalesced
@@ -154,10 +156,10 @@ cudaError_t launch_frames_to_u8(const FramesParams& p, cudaStream_t stream)
 #define DIT_FRAMES_CASE(CC)                                                                                  \
     if (p.C == CC) {                                                                                         \
         if (p.layout == 0)                                                                                   \
-            frames_vec_kernel<CC, 0><<<grid, kCtaThreads, 0, stream>>>(p.x, p.out, p.T, p.H, p.W, items);    \
-        else                                                                                                 \
-            frames_vec_kernel<CC, 1><<<grid, kCtaThreads, 0, stream>>>(p.x, p.out, p.T, p.H, p.W, items);    \
-        return cudaGetLastError();                                                                           \
+            return launch_kernel(frames_vec_kernel<CC, 0>, grid, kCtaThreads, 0, stream, p.x, p.out, p.T, p.H, \
+                                 p.W, items);                                                                \
+        return launch_kernel(frames_vec_kernel<CC, 1>, grid, kCtaThreads, 0, stream, p.x, p.out, p.T, p.H, p.W, \
+                             items);                                                                         \
     }
         DIT_FRAMES_CASE(1)
         DIT_FRAMES_CASE(3)
@@ -165,9 +167,8 @@ cudaError_t launch_frames_to_u8(const FramesParams& p, cudaStream_t stream)
 #undef DIT_FRAMES_CASE
     }
     const int64_t items = p.B * p.C * p.T * p.H * p.W;
-    frames_scalar_kernel<<<grid_for(items), kCtaThreads, 0, stream>>>(p.x, p.out, p.C, p.T, p.H, p.W, p.layout,
-                                                                     items);
-    return cudaGetLastError();
+    return launch_kernel(frames_scalar_kernel, grid_for(items), kCtaThreads, 0, stream, p.x, p.out, p.C, p.T, p.H,
+                         p.W, (int32_t)p.layout, items);
 }
 
 }  // namespace dit

@@ -3,29 +3,35 @@
 // DiT", "Key takeaways", bullet 2: the residual update is one of the fused
 // operators).
 //
-// One warp per valid row; each lane streams U 16-byte vectors of x and y per
-// step (all loads of a step are issued before any arithmetic), adds
-// gate * y with one fp32 FMA per element and rounds once.  The gate vector
-// (bf16, or fp32 as the modulation head may emit it) is read through the
-// read-only path: it is shared by every row of a sequence and stays in L1/L2.
-// HBM traffic: 6 bytes per element (x, y in; out out).
+// One warp per valid row in CTAs of 4 warps; each lane streams UNR vectors of
+// x and y per step (all loads of a step are issued before any arithmetic),
+// adds gate * y with one fp32 FMA per element and rounds once.  The gate
+// vector (bf16, or fp32 as the modulation head may emit it) is read through
+// the read-only path: it is shared by every row of a sequence and stays in
+// L1/L2.  With a bf16 gate and rows on 32-byte boundaries a lane moves 32
+// bytes per access (2 vectors in flight): 308 us on batched varlen (hidden
+// 5120, 2.15 GB) against 314 us with 16-byte accesses, and 22.5 against 24.6
+// us on one rank's slice of the long video (7,736 rows of 3072).  An fp32
+// gate keeps 16-byte activation accesses, so that a lane's share of the gate
+// is one contiguous 32-byte piece.  HBM traffic: 6 bytes per element (x, y
+// in; out out).
 #include "common.cuh"
 #include "launch.h"
 
 namespace dit {
 namespace {
 
-#ifndef DIT_EW_UNROLL
-#define DIT_EW_UNROLL 4
-#endif
-constexpr int kUnroll = DIT_EW_UNROLL;  // 16-byte vectors per lane and input in flight
+constexpr int kResWarps = 4;  // rows (warps) per CTA
 
-template <bool F32>
-__global__ void __launch_bounds__(kCtaThreads)
+template <int NW, int UNR, bool F32>
+__global__ void __launch_bounds__(kResWarps * kWarp)
 gated_residual_kernel(const GatedParams p)
 {
+    constexpr int EPV = 2 * NW;
+    constexpr int NG = NW < 4 ? NW : 4;  // words per read of the gate
+    grid_dependency_wait();
     const int lane = threadIdx.x & (kWarp - 1);
-    const int v = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int v = blockIdx.x * kResWarps + (threadIdx.x >> 5);
     RowSlot s;
     if (!map_valid_row(v, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs,
                        p.pk.num_rows_padded, lane, s))
@@ -34,33 +40,33 @@ gated_residual_kernel(const GatedParams p)
     const uint16_t* yr = p.y + (int64_t)s.row * p.y_row_stride;
     const int64_t goff = (int64_t)s.seq * p.gate_seq_stride;
     uint16_t* orow = p.out + (int64_t)s.row * p.out_row_stride;
-    const int nvec = p.hidden / 8;
+    const int nvec = p.hidden / EPV;
 
-    for (int c0 = 0; c0 < nvec; c0 += kWarp * kUnroll) {
-        uint4 xv[kUnroll], yv[kUnroll];
-        Vec8Raw<F32> gv[kUnroll];
+    for (int c0 = 0; c0 < nvec; c0 += kWarp * UNR) {
+        uint32_t xv[UNR][NW], yv[UNR][NW];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < UNR; ++u) {
             const int j = c0 + u * kWarp + lane;
             if (j < nvec) {
-                xv[u] = ld_stream(xr + 8 * j);
-                yv[u] = ld_stream(yr + 8 * j);
-                gv[u] = vec8_load<F32>(p.gate, goff + 8 * j);
+                ld_stream_words<NW>(xr + EPV * j, xv[u]);
+                ld_stream_words<NW>(yr + EPV * j, yv[u]);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < UNR; ++u) {
             const int j = c0 + u * kWarp + lane;
             if (j < nvec) {
-                const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-                const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
-                f32x2 g[4];
-                vec8_unpack<F32>(gv[u], g);
-                uint32_t o[4];
+                uint32_t o[NW];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    o[e] = f2_to_bf16x2(f2_fma(g[e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
-                st_stream(orow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
+                for (int h = 0; h < NW / NG; ++h) {
+                    f32x2 g[NG];
+                    vec_pairs<F32, NG>(p.gate, goff + EPV * j + 2 * NG * h, g);
+#pragma unroll
+                    for (int e = 0; e < NG; ++e)
+                        o[NG * h + e] = f2_to_bf16x2(
+                            f2_fma(g[e], f2_from_bf16x2(yv[u][NG * h + e]), f2_from_bf16x2(xv[u][NG * h + e])));
+                }
+                st_stream_words<NW>(orow + EPV * j, o);
             }
         }
     }
@@ -70,12 +76,14 @@ gated_residual_kernel(const GatedParams p)
 
 cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream)
 {
-    const unsigned grid = (unsigned)((p.pk.num_rows_padded + kWarpsPerCta - 1) / kWarpsPerCta);
+    const unsigned grid = (unsigned)((p.pk.num_rows_padded + kResWarps - 1) / kResWarps);
+    const dim3 block(kResWarps * kWarp);
     if (p.gate_f32)
-        gated_residual_kernel<true><<<grid, kCtaThreads, 0, stream>>>(p);
-    else
-        gated_residual_kernel<false><<<grid, kCtaThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_kernel(gated_residual_kernel<4, 4, true>, grid, block, 0, stream, p);
+    const bool wide = aligned32(p.x) && aligned32(p.y) && aligned32(p.out) && p.hidden % 16 == 0 &&
+                      p.x_row_stride % 16 == 0 && p.y_row_stride % 16 == 0 && p.out_row_stride % 16 == 0;
+    return wide ? launch_kernel(gated_residual_kernel<8, 2, false>, grid, block, 0, stream, p)
+                : launch_kernel(gated_residual_kernel<4, 4, false>, grid, block, 0, stream, p);
 }
 
 }  // namespace dit

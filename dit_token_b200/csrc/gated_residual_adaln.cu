@@ -11,52 +11,67 @@
 // norm written once: 8 bytes per element instead of the 10 of the unfused
 // pair.
 //
-// Layout as in adaln_modulate.cu: a team of TEAM warps owns a row and keeps
-// the rounded residual in registers (VPT 16-byte vectors per lane); one-pass
-// moments for the statistics, packed fp32 pairs for the arithmetic.  gate,
-// shift and scale are bf16, or all three fp32.  One short-lived CTA per two
-// to four rows: a persistent form (each team a fixed run of rows, the
-// vectors staged once per CTA in shared memory as fp32) measured slower,
-// 569 against 455 us on batched varlen (hidden 5120) and 322 against 234 us
-// on 61,888 rows of hidden 3072, even with fp32 vectors (591 against 527 us).
+// Layout: one short-lived CTA per row, a team of TEAM warps (1-8) that keeps
+// the rounded residual in registers (VPT vectors of NW words per lane);
+// one-pass moments per warp, merged across the team through shared memory
+// behind one barrier; packed fp32 pairs for the arithmetic.  gate, shift and
+// scale are bf16, or all three fp32.  The access width per lane and the team
+// size come from a sweep over both (batched varlen, hidden 5120, L2 clean,
+// the B200's measured copy bandwidth 6458 GB/s):
+//  * bf16 vectors: 32-byte accesses, the smallest team that holds the row in
+//    at most 3 vectors per lane (5120: 4 warps, 3072 and 2048: 2 warps):
+//    424.9 us (104 %), against 456.7 us for the earlier kernel (16-byte
+//    accesses, 2-4 rows per 8-warp CTA); 61,888 rows of 3072: 227.4 against
+//    235.5 us;
+//  * fp32 vectors: a lane's share of each fp32 vector is contiguous only
+//    with 8- or 16-byte activation accesses (with 32-byte ones each warp
+//    load instruction spans 2 KB of the vector: 56-66 %).
+// A persistent form (each team a fixed run of rows, the vectors staged once
+// per CTA in shared memory as fp32) measured slower: 569 against 455 us on
+// batched varlen, 322 against 234 us on 61,888 rows of 3072, and 591 against
+// 527 us with fp32 vectors.
 #include "common.cuh"
 #include "launch.h"
 
 namespace dit {
 namespace {
 
-template <int VPT, int TEAM, bool F32>
-__global__ void __launch_bounds__(kCtaThreads, MinCtas<VPT, 2>::value)
+template <int VPT, int NW, int TEAM, bool F32>
+__global__ void __launch_bounds__(TEAM * kWarp)
 gated_residual_adaln_kernel(const FusedParams p)
 {
-    constexpr int kRowsPerCta = kWarpsPerCta / TEAM;
+    constexpr int EPV = 2 * NW;                  // elements per vector
+    constexpr int NG = NW < 4 ? NW : 4;          // words per group of per-sequence vector reads
     constexpr int kTeamThreads = TEAM * kWarp;
-    __shared__ Moments red[kWarpsPerCta];
+    __shared__ Moments red[TEAM];
+    grid_dependency_wait();
 
     const int lane = threadIdx.x & (kWarp - 1);
     const int warp = threadIdx.x >> 5;
-    const int team = warp / TEAM;
-    const int tt = (warp % TEAM) * kWarp + lane;
-    const int v = blockIdx.x * kRowsPerCta + team;
+    const int tt = threadIdx.x;
     RowSlot s;
-    const bool active = map_valid_row(v, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs,
-                                      p.pk.num_rows_padded, lane, s);
-    if (!active)
-        return;  // the whole team leaves: its barriers involve only its own warps
-    const int nvec = p.hidden / 8;
+    if (!map_valid_row(blockIdx.x, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded,
+                       lane, s))
+        return;  // uniform over the CTA: every warp maps the same row
+    const int nvec = p.hidden / EPV;
 
     // residual update, rounded once, kept packed
-    uint4 rv[VPT];
+    uint32_t rv[VPT][NW];
     {
-        uint4 xv[VPT], yv[VPT];
+        uint32_t xv[VPT][NW], yv[VPT][NW];
         const uint16_t* xr = p.x + (int64_t)s.row * p.x_row_stride;
         const uint16_t* yr = p.y + (int64_t)s.row * p.y_row_stride;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int j = i * kTeamThreads + tt;
-            const bool in = j < nvec;
-            xv[i] = in ? ld_stream(xr + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
-            yv[i] = in ? ld_stream(yr + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+            if (j < nvec) {
+                ld_stream_words<NW>(xr + EPV * j, xv[i]);
+                ld_stream_words<NW>(yr + EPV * j, yv[i]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < NW; ++e)
+                    xv[i][e] = yv[i][e] = 0u;
+            }
         }
         const int64_t goff = (int64_t)s.seq * p.gate_seq_stride;
         uint16_t* res = p.res_out + (int64_t)s.row * p.res_row_stride;
@@ -64,53 +79,50 @@ gated_residual_adaln_kernel(const FusedParams p)
         for (int i = 0; i < VPT; ++i) {
             const int j = i * kTeamThreads + tt;
             if (j < nvec) {
-                f32x2 g[4];
-                vec8_pairs<F32>(p.gate, goff + 8 * j, g);
-                const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
-                const uint32_t yw[4] = {yv[i].x, yv[i].y, yv[i].z, yv[i].w};
-                uint32_t o[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    o[e] = f2_to_bf16x2(f2_fma(g[e], f2_from_bf16x2(yw[e]), f2_from_bf16x2(xw[e])));
-                rv[i] = make_uint4(o[0], o[1], o[2], o[3]);
-                st_stream(res + 8 * j, rv[i]);
+                for (int h = 0; h < NW / NG; ++h) {
+                    f32x2 g[NG];
+                    vec_pairs<F32, NG>(p.gate, goff + EPV * j + 2 * NG * h, g);
+#pragma unroll
+                    for (int e = 0; e < NG; ++e)
+                        rv[i][NG * h + e] = f2_to_bf16x2(
+                            f2_fma(g[e], f2_from_bf16x2(yv[i][NG * h + e]), f2_from_bf16x2(xv[i][NG * h + e])));
+                }
+                st_stream_words<NW>(res + EPV * j, rv[i]);
             } else {
-                rv[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int e = 0; e < NW; ++e)
+                    rv[i][e] = 0u;
             }
         }
     }
 
     // LN statistics of the stored residual: shifted sums, merged as moments
-    const float k = bf16_lo(rv[0].x);
+    const float k = bf16_lo(rv[0][0]);
     const f32x2 kk = f2_make(k, k);
     f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
     float cnt = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int j = i * kTeamThreads + tt;
-        if (j < nvec) {
-            const uint32_t w[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
+        if (i * kTeamThreads + tt < nvec) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const f32x2 d = f2_sub(f2_from_bf16x2(w[e]), kk);
+            for (int e = 0; e < NW; ++e) {
+                const f32x2 d = f2_sub(f2_from_bf16x2(rv[i][e]), kk);
                 s2 = f2_add(s2, d);
                 q2 = f2_fma(d, d, q2);
             }
-            cnt += 8.f;
+            cnt += (float)EPV;
         }
     }
-    float s0, s1, q0, q1;
-    f2_split(s2, s0, s1);
-    f2_split(q2, q0, q1);
-    Moments m = moments_warp(moments_from_sums(cnt, k, s0 + s1, q0 + q1));
+    Moments m = moments_warp(moments_from_sums(cnt, k, s2.x + s2.y, q2.x + q2.y));
     if (TEAM > 1) {
         if (lane == 0)
             red[warp] = m;
-        team_barrier<TEAM>(team);
-        m = red[team * TEAM];
+        __syncthreads();
+        m = red[0];
 #pragma unroll
         for (int w = 1; w < TEAM; ++w)
-            m = moments_merge(m, red[team * TEAM + w]);
+            m = moments_merge(m, red[w]);
     }
     const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);  // as in adaln_modulate.cu
     const f32x2 r2 = f2_make(rstd, rstd);
@@ -124,71 +136,74 @@ gated_residual_adaln_kernel(const FusedParams p)
     for (int i = 0; i < VPT; ++i) {
         const int j = i * kTeamThreads + tt;
         if (j < nvec) {
-            f32x2 hv[4], cv[4];
-            vec8_pairs<F32>(p.shift, moff + 8 * j, hv);
-            vec8_pairs<F32>(p.scale, moff + 8 * j, cv);
-            const uint32_t rw[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
-            uint32_t o[4];
+            uint32_t o[NW];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const f32x2 t = f2_fma(f2_from_bf16x2(rw[e]), r2, b2);
-                o[e] = f2_to_bf16x2(f2_fma(t, f2_add(cv[e], one2), hv[e]));
+            for (int h = 0; h < NW / NG; ++h) {
+                f32x2 hv[NG], cv[NG];
+                vec_pairs<F32, NG>(p.shift, moff + EPV * j + 2 * NG * h, hv);
+                vec_pairs<F32, NG>(p.scale, moff + EPV * j + 2 * NG * h, cv);
+#pragma unroll
+                for (int e = 0; e < NG; ++e) {
+                    const f32x2 t = f2_fma(f2_from_bf16x2(rv[i][NG * h + e]), r2, b2);
+                    o[NG * h + e] = f2_to_bf16x2(f2_fma(t, f2_add(cv[e], one2), hv[e]));
+                }
             }
-            st_stream(nrow + 8 * j, make_uint4(o[0], o[1], o[2], o[3]));
+            st_stream_words<NW>(nrow + EPV * j, o);
         }
     }
 }
 
-template <int TEAM, int VPT>
-void launch_one(const FusedParams& p, cudaStream_t stream)
+template <int VPT, int NW, int TEAM, bool F32>
+cudaError_t launch_one(const FusedParams& p, cudaStream_t stream)
 {
-    const int rows_per_cta = kWarpsPerCta / TEAM;
-    const unsigned grid = (unsigned)((p.pk.num_rows_padded + rows_per_cta - 1) / rows_per_cta);
-    if (p.mod_f32)
-        gated_residual_adaln_kernel<VPT, TEAM, true><<<grid, kCtaThreads, 0, stream>>>(p);
-    else
-        gated_residual_adaln_kernel<VPT, TEAM, false><<<grid, kCtaThreads, 0, stream>>>(p);
+    const unsigned grid = (unsigned)p.pk.num_rows_padded;  // one row per CTA
+    return launch_kernel(gated_residual_adaln_kernel<VPT, NW, TEAM, F32>, grid, TEAM * kWarp, 0, stream, p);
 }
 
-template <int TEAM>
-cudaError_t launch_team(const FusedParams& p, int vpt, cudaStream_t stream)
+// VPT (1..MAXV) as a template argument.
+template <int NW, int TEAM, bool F32, int MAXV, int V = 1>
+cudaError_t launch_vpt(const FusedParams& p, int vpt, cudaStream_t stream)
 {
-    switch (vpt) {
-    case 1: launch_one<TEAM, 1>(p, stream); break;
-    case 2: launch_one<TEAM, 2>(p, stream); break;
-    case 3: launch_one<TEAM, 3>(p, stream); break;
-    case 4: launch_one<TEAM, 4>(p, stream); break;
-    case 5: launch_one<TEAM, 5>(p, stream); break;
-    case 6: launch_one<TEAM, 6>(p, stream); break;
-    case 7: launch_one<TEAM, 7>(p, stream); break;
-    case 8: launch_one<TEAM, 8>(p, stream); break;
-    default: return cudaErrorInvalidValue;
+    if constexpr (V > MAXV) {
+        return cudaErrorInvalidValue;
+    } else {
+        if (vpt == V)
+            return launch_one<V, NW, TEAM, F32>(p, stream);
+        return launch_vpt<NW, TEAM, F32, MAXV, V + 1>(p, vpt, stream);
     }
-    return cudaGetLastError();
+}
+
+// The smallest team of 1, 2, 4 or 8 warps that holds the row in at most
+// MAXV vectors of NW words per lane (the widest rows: 8 warps, up to 8
+// vectors).
+template <int NW, bool F32, int MAXV>
+cudaError_t launch_width(const FusedParams& p, cudaStream_t stream)
+{
+    const int nvec = p.hidden / (2 * NW);
+    auto vpt_for = [&](int team) { return (nvec + team * kWarp - 1) / (team * kWarp); };
+    if (vpt_for(1) <= MAXV)
+        return launch_vpt<NW, 1, F32, MAXV>(p, vpt_for(1), stream);
+    if (vpt_for(2) <= MAXV)
+        return launch_vpt<NW, 2, F32, MAXV>(p, vpt_for(2), stream);
+    if (vpt_for(4) <= MAXV)
+        return launch_vpt<NW, 4, F32, MAXV>(p, vpt_for(4), stream);
+    return launch_vpt<NW, 8, F32, 8>(p, vpt_for(8), stream);
 }
 
 }  // namespace
 
-// Team size: the smallest of 2, 4, 8 warps that holds the row in at most 8
-// vectors per lane (hidden 2048 -> 2 warps, 3072 -> 2, 5120 -> 4).  A single
-// warp per row was measured slower on short rows (hidden 2048: 36.9 against
-// 29.9 us for 8192 rows), and at most 4 vectors per lane slower on long ones
-// (hidden 5120: 568 against 456 us).
+// Access width: bf16 vectors take 32-byte accesses when all four row buffers
+// are 32-byte aligned and hidden and every row stride are multiples of 16
+// elements (each row then starts on a 32-byte boundary), else 16-byte ones;
+// fp32 vectors take 16-byte accesses (teams of at most 5 vectors per lane).
 cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream)
 {
-    const int nvec = p.hidden / 8;
-    for (int team = 2; team <= kWarpsPerCta; team *= 2) {
-        const int per = team * kWarp;
-        const int vpt = (nvec + per - 1) / per;
-        if (vpt > 8)
-            continue;
-        switch (team) {
-        case 2: return launch_team<2>(p, vpt, stream);
-        case 4: return launch_team<4>(p, vpt, stream);
-        default: return launch_team<8>(p, vpt, stream);
-        }
-    }
-    return cudaErrorInvalidValue;  // hidden > kMaxAdalnHidden, rejected by the ABI first
+    if (p.mod_f32)
+        return launch_width<4, true, 5>(p, stream);
+    const bool wide = aligned32(p.x) && aligned32(p.y) && aligned32(p.res_out) && aligned32(p.norm_out) &&
+                      p.hidden % 16 == 0 && p.x_row_stride % 16 == 0 && p.y_row_stride % 16 == 0 &&
+                      p.res_row_stride % 16 == 0 && p.norm_row_stride % 16 == 0;
+    return wide ? launch_width<8, false, 3>(p, stream) : launch_width<4, false, 5>(p, stream);
 }
 
 }  // namespace dit

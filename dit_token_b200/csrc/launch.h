@@ -4,9 +4,45 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 namespace dit {
+
+// Programmatic dependent launch.  Every kernel of the library starts with
+// grid_dependency_wait() (common.cuh) before its first global-memory access
+// -- the packing descriptors included -- and then lets its own dependents
+// launch.  So each launch may carry the programmatic-serialization attribute:
+// when the previous kernel on the stream lets it, this kernel's CTAs are
+// placed and resident while that kernel drains, and start the moment it
+// completes (its writes visible), instead of after a full launch gap.  A
+// kernel launched after one that does not take part simply starts when that
+// one completes, as without the attribute.  DIT_PDL=0 at build time launches
+// plainly (for comparison).
+#ifndef DIT_PDL
+#define DIT_PDL 1
+#endif
+
+// A 32-byte boundary (the 256-bit row accesses need one).
+inline bool aligned32(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0; }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = DIT_PDL ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct Packing {
     const int32_t* cu_seqlens;

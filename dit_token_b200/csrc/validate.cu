@@ -10,9 +10,13 @@ namespace {
 __global__ void validate_seqlens_kernel(const int32_t* __restrict__ cs, const int32_t* __restrict__ cp,
                                         int B, long long rows_padded, int32_t* flag)
 {
-    // One warp; lanes stride over sequences and the first failure wins.
+    // One warp; lanes stride over sequences and the first failure wins.  The
+    // leading entries are checked whatever the sequence count, so an empty
+    // batch whose descriptor does not start at 0 is reported too.
+    constexpr int kNone = 0x7fffffff;
+    grid_dependency_wait();
     const int lane = threadIdx.x;
-    int first_bad = B;  // sentinel: no failure
+    int first_bad = kNone;
     if (lane == 0 && (cs[0] != 0 || cp[0] != 0))
         first_bad = 0;
     for (int b = lane; b < B; b += kWarp) {
@@ -25,8 +29,8 @@ __global__ void validate_seqlens_kernel(const int32_t* __restrict__ cs, const in
     for (int o = 16; o >= 1; o >>= 1)
         first_bad = min(first_bad, __shfl_xor_sync(0xffffffffu, first_bad, o));
     if (lane == 0) {
-        flag[0] = first_bad < B ? 1 : 0;
-        flag[1] = first_bad < B ? first_bad : -1;
+        flag[0] = first_bad != kNone ? 1 : 0;
+        flag[1] = first_bad != kNone ? first_bad : -1;
     }
 }
 
@@ -35,9 +39,8 @@ __global__ void validate_seqlens_kernel(const int32_t* __restrict__ cs, const in
 cudaError_t launch_validate_seqlens(const Packing& pk, int64_t num_rows_padded, int32_t* flag,
                                     cudaStream_t stream)
 {
-    validate_seqlens_kernel<<<1, kWarp, 0, stream>>>(pk.cu_seqlens, pk.cu_seqlens_padded, pk.num_seqs,
-                                                     (long long)num_rows_padded, flag);
-    return cudaGetLastError();
+    return launch_kernel(validate_seqlens_kernel, 1, kWarp, 0, stream, pk.cu_seqlens, pk.cu_seqlens_padded,
+                         (int)pk.num_seqs, (long long)num_rows_padded, flag);
 }
 
 }  // namespace dit

@@ -40,8 +40,17 @@
  *             q and k are always updated in place.
  *             Partial overlap is undefined.
  * Stream      `stream` is a cudaStream_t (NULL = the legacy default stream).
- *             Calls only enqueue work: they never synchronize, allocate or
- *             keep state, and are safe to call from several host threads.
+ *             Calls only enqueue work: they never synchronize or allocate,
+ *             and are safe to call from several host threads.  The only
+ *             state is per host thread: the last CUDA error and a copy of
+ *             the last rotary frequency table (reused while theta, head_dim
+ *             and the sections stay the same).
+ * Launches    every kernel is launched with programmatic stream
+ *             serialization and waits for the previous kernel on the stream
+ *             to complete before its first memory access, so back-to-back
+ *             calls overlap launch latency (not work); this is invisible to
+ *             the caller, and a kernel launched after one of these starts
+ *             as usual unless it opts in the same way.
  * Errors      argument errors are returned BEFORE anything is launched; a
  *             failed launch returns DIT_ERR_CUDA (dit_last_cuda_error gives
  *             the CUDA error code seen by this thread).  No entry point traps
@@ -139,7 +148,9 @@ DIT_API dit_status dit_qk_rmsnorm_rope_ex(void* q, int64_t q_row_stride, void* k
  * sequence b, and take that sequence's positions: with rope_grid[b] =
  * (T, H, W), whole-sequence rows below T*H*W are 3D, the rest 1D counted from
  * the end of the grid.  pos_offset: device int32 [num_seqs] (>= 0), or NULL
- * (every offset 0: the _ex call).  Ignored when rope_mode is DIT_ROPE_NONE. */
+ * (every offset 0: the _ex call).  Ignored when rope_mode is DIT_ROPE_NONE.
+ * The offsets are trusted like cu_seqlens: a negative entry, outside the
+ * documented range, is read as 0 (no fault and no flag). */
 DIT_API dit_status dit_qk_rmsnorm_rope_shard(void* q, int64_t q_row_stride, void* k, int64_t k_row_stride,
                                              const void* q_weight, const void* k_weight,
                                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,
@@ -281,7 +292,8 @@ DIT_API dit_status dit_frames_to_u8(const float* x, int64_t batch, int64_t chann
  * Writes flag[0] = 0 if cu_seqlens[0] == 0, cu_seqlens_padded[0] == 0, both
  * are non-decreasing, every valid length fits its padded slot and
  * cu_seqlens_padded[num_seqs] <= num_rows_padded; otherwise flag[0] = 1 and
- * flag[1] = the first offending sequence index.  flag: device int32[2].  The
+ * flag[1] = the first offending sequence index (0 also when a leading entry
+ * is not 0, even for num_seqs == 0).  flag: device int32[2].  The
  * kernel never traps; the host reads the flag when it chooses to (e.g. with
  * cudaMemcpy after the stream) and maps 1 to DIT_ERR_SEQLENS. */
 DIT_API dit_status dit_validate_seqlens(const int32_t* cu_seqlens, const int32_t* cu_seqlens_padded,

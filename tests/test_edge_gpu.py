@@ -148,7 +148,7 @@ def test_fused_qkv_slices_and_wide_out_stride():
     assert torch.all(wide[:, :w.hidden].view(torch.int16) == W.SENTINEL)
 
 
-@pytest.mark.parametrize("hidden", [8, 256, 264, 2048, 2056, 3072, 4096, 5120, 8192, 16384])
+@pytest.mark.parametrize("hidden", [8, 256, 264, 2048, 2056, 3072, 4096, 5120, 6136, 6144, 6152, 8192, 16384])
 def test_adaln_every_team_shape(hidden):
     w = W.custom("adaln", (13, 6), (16, 8), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
                  inner=8, seed=hidden)
@@ -162,6 +162,35 @@ def test_adaln_every_team_shape(hidden):
     r_ref, n_ref = P.oracle_fused(w, inp, rows)
     P.assert_close(P.gather_rows(res, rows), r_ref[rows], f"fused residual {hidden}")
     P.assert_close(P.gather_rows(norm, rows), n_ref[rows], f"fused norm {hidden}")
+
+
+@pytest.mark.parametrize("offset", [0, 8, 16])
+def test_adaln_row_alignment(offset):
+    """adaLN reads and writes 32 bytes per lane access when every row starts
+    on a 32-byte boundary and 16 bytes otherwise: rows starting `offset`
+    elements into a wider buffer (8: 16-byte aligned only) agree with the
+    oracle either way, in place too."""
+    w = W.custom("adaln_al", (300, 77), (304, 80), hidden=3072, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=41)
+    C, rows = w.hidden, w.valid_rows()
+    inp = W.adaln_inputs(w)
+    ref = P.oracle_adaln(w, inp, rows)
+    cs, cp, _ = P.device_packing(w)
+    mod = inp["mod"].cuda()
+    buf = W.sentinel_like((inp["x"].shape[0], C + 32)).cuda()
+    buf[:, offset:offset + C] = inp["x"].cuda()
+    x = W.rows_view(buf)[:, offset:offset + C]
+    out = W.sentinel_like((inp["x"].shape[0], C + 32)).cuda()
+    o = W.rows_view(out)[:, offset:offset + C]
+    dit.dit_adaln_modulate(x, mod[:, 0], mod[:, 1], cs, cp, out=o, eps=w.eps)
+    dit.dit_adaln_modulate(x, mod[:, 0], mod[:, 1], cs, cp, out=x, eps=w.eps)   # in place
+    torch.cuda.synchronize()
+    for name, t in (("out", out), ("in place", buf)):
+        got = P.gather_rows(t[:, offset:offset + C].contiguous(), rows)
+        P.assert_close(got, ref[rows], f"adaln offset {offset} {name}")
+        # columns outside the row slice are untouched
+        assert torch.all(t[:, :offset].view(torch.int16) == W.SENTINEL)
+        assert torch.all(t[:, offset + C:].view(torch.int16) == W.SENTINEL)
 
 
 def test_swiglu_extreme_activations():
@@ -217,6 +246,15 @@ def test_malformed_device_descriptors_are_skipped_and_flagged():
     bad2 = dit.dit_validate_seqlens(cs2, cp2, 16)
     torch.cuda.synchronize()
     assert good.tolist()[0] == 0 and bad2.tolist() == [1, 1]
+    # an empty batch is still checked for its leading entries
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    one = torch.ones(1, dtype=torch.int32, device="cuda")
+    empty_ok = dit.dit_validate_seqlens(z, z, 0)
+    empty_bad = dit.dit_validate_seqlens(one, z, 0)
+    empty_bad_p = dit.dit_validate_seqlens(z, one, 4)
+    torch.cuda.synchronize()
+    assert empty_ok.tolist() == [0, -1]
+    assert empty_bad.tolist() == [1, 0] and empty_bad_p.tolist() == [1, 0]
 
 
 def test_check_seqlens_raises_on_malformed_descriptors():
@@ -301,3 +339,27 @@ def test_small_rows_many_sequences(mode, sliced):
     keep = P.untouched_rows(w)
     P.assert_untouched(q, inp["q"], keep, "small rows q")
     P.assert_untouched(k, inp["k"], keep, "small rows k")
+
+
+def test_negative_position_offset_reads_as_zero():
+    """pos_offset entries are documented as >= 0; a negative one is read as 0
+    (whole-sequence positions from the slice's own first row), including with
+    an empty grid, and nothing outside the valid rows is written."""
+    w = W.custom("negoff", (40, 30), (48, 32), hidden=256, num_q_heads=1, num_k_heads=1, head_dim=128, inner=64,
+                 grids=((1, 4, 5), (0, 0, 7)), sections=(44, 42, 42), seed=31)
+    inp = W.qk_inputs(w)
+    cs, cp, grid = P.device_packing(w)
+    outs = []
+    for offs in ([0, 0], [-5, -1000]):
+        q, k = inp["q"].cuda(), inp["k"].cuda()
+        dit.dit_qk_rmsnorm_rope(W.rows_view(q), W.rows_view(k), inp["q_weight"].cuda(), inp["k_weight"].cuda(),
+                                cs, cp, num_q_heads=1, num_k_heads=1, head_dim=128, rope_grid=grid,
+                                sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
+                                pos_offset=torch.tensor(offs, dtype=torch.int32, device="cuda"))
+        outs.append((q, k))
+    torch.cuda.synchronize()
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    keep = P.untouched_rows(w)
+    P.assert_untouched(outs[1][0], inp["q"], keep, "negative offset q")
+    P.assert_untouched(outs[1][1], inp["k"], keep, "negative offset k")

@@ -68,7 +68,12 @@ def test_f32_modulation_many_short_sequences():
 
 
 @pytest.mark.parametrize("hidden", [264, 5120, 8192])
-def test_bf16_valued_f32_vectors_match_the_bf16_path_bitwise(hidden):
+def test_bf16_valued_f32_vectors_match_the_bf16_path(hidden):
+    """fp32 vectors holding bf16 values give the bf16 path's results: the
+    element-wise residuals bit for bit; the normalizations (whose row
+    statistics the two paths sum in different lane layouts -- they use
+    different access widths) within the tolerance and almost all bit for
+    bit."""
     w = W.custom("same", (37, 5, 90), (40, 8, 96), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
                  inner=8, seed=7)
     cs, cp, _ = P.device_packing(w)
@@ -79,14 +84,20 @@ def test_bf16_valued_f32_vectors_match_the_bf16_path_bitwise(hidden):
     a = dit.dit_adaln_modulate(x, m16[:, 0], m16[:, 1], cs, cp, eps=w.eps)
     b = dit.dit_adaln_modulate(x, m32[:, 0], m32[:, 1], cs, cp, eps=w.eps)
     rows = torch.from_numpy(w.valid_rows()).cuda()
-    assert torch.equal(a[rows].view(torch.int16), b[rows].view(torch.int16))
+
+    def close(u, v, what):
+        ub, vb = u[rows].view(torch.int16), v[rows].view(torch.int16)
+        P.assert_close(ub.cpu().numpy().view(np.uint16), vb.cpu().numpy().view(np.uint16), what)
+        assert (ub == vb).float().mean().item() >= 0.999, what
+
+    close(a, b, "adaln")
     a = dit.dit_gated_residual(x, y, m16[:, 2], cs, cp)
     b = dit.dit_gated_residual(x, y, m32[:, 2], cs, cp)
     assert torch.equal(a[rows].view(torch.int16), b[rows].view(torch.int16))
     ra, na = dit.dit_gated_residual_adaln(x, y, m16[:, 2], m16[:, 3], m16[:, 4], cs, cp, eps=w.eps)
     rb, nb = dit.dit_gated_residual_adaln(x, y, m32[:, 2], m32[:, 3], m32[:, 4], cs, cp, eps=w.eps)
     assert torch.equal(ra[rows].view(torch.int16), rb[rows].view(torch.int16))
-    assert torch.equal(na[rows].view(torch.int16), nb[rows].view(torch.int16))
+    close(na, nb, "fused norm")
 
 
 def test_f32_modulation_batched_varlen_sampled():
