@@ -279,6 +279,38 @@ __device__ __forceinline__ void vec8_pairs(const void* base, int64_t elem, f32x2
     vec8_unpack<F32>(vec8_load<F32>(base, elem), v);
 }
 
+// 32 bytes of a per-sequence vector (16 bf16 or 8 fp32 elements) through the
+// read-only path in one 256-bit load (sm_100); the address must be 32-byte
+// aligned.  With a lane's share of a vector this wide, a warp's vector loads
+// cover contiguous memory, so each 128-byte line is fetched once per load
+// instruction instead of twice.
+__device__ __forceinline__ void ld_vec32(const void* p, uint32_t (&w)[8])
+{
+    asm("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+        : "l"(p));
+}
+
+// NP pairs of a per-sequence vector at element `elem` as fp32 pairs, read 32
+// bytes at a time: bf16 takes NP = 8 (16 elements), fp32 NP = 4 (8 elements).
+template <bool F32, int NP>
+__device__ __forceinline__ void vec_pairs_wide(const void* base, int64_t elem, f32x2 (&v)[NP])
+{
+    static_assert(NP == (F32 ? 4 : 8), "32 bytes: 16 bf16 or 8 fp32 elements");
+    uint32_t w[8];
+    if constexpr (F32) {
+        ld_vec32(static_cast<const float*>(base) + elem, w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            v[e] = make_float2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+    } else {
+        ld_vec32(static_cast<const uint16_t*>(base) + elem, w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            v[e] = f2_from_bf16x2(w[e]);
+    }
+}
+
 // NP consecutive pairs (2 * NP elements, NP = 2 or 4) of a per-sequence
 // vector starting at element `elem`, as fp32 pairs: one 8- or 16-byte load
 // (bf16) or one or two 16-byte loads (fp32) through the read-only path.

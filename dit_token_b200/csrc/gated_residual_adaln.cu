@@ -25,7 +25,8 @@
 //    235.5 us;
 //  * fp32 vectors: a lane's share of each fp32 vector is contiguous only
 //    with 8- or 16-byte activation accesses (with 32-byte ones each warp
-//    load instruction spans 2 KB of the vector: 56-66 %).
+//    load instruction spans 2 KB of the vector: 56-66 %); 16-byte ones with
+//    the vectors read 32 bytes at a time: 456.7 us (97 %).
 // A persistent form (each team a fixed run of rows, the vectors staged once
 // per CTA in shared memory as fp32) measured slower: 569 against 455 us on
 // batched varlen, 322 against 234 us on 61,888 rows of 3072, and 591 against
@@ -36,12 +37,25 @@
 namespace dit {
 namespace {
 
-template <int VPT, int NW, int TEAM, bool F32>
+// A group of NG pairs of a per-sequence vector: 32-byte reads (WV: 8 bf16 or
+// 4 fp32 pairs) or 8/16-byte ones.
+template <bool F32, int NG, bool WV>
+__device__ __forceinline__ void seq_pairs(const void* base, int64_t elem, f32x2 (&v)[NG])
+{
+    if constexpr (WV)
+        vec_pairs_wide<F32, NG>(base, elem, v);
+    else
+        vec_pairs<F32, NG>(base, elem, v);
+}
+
+template <int VPT, int NW, int TEAM, bool F32, bool WV = false>
 __global__ void __launch_bounds__(TEAM * kWarp)
 gated_residual_adaln_kernel(const FusedParams p)
 {
     constexpr int EPV = 2 * NW;                  // elements per vector
-    constexpr int NG = NW < 4 ? NW : 4;          // words per group of per-sequence vector reads
+    // words per group of per-sequence vector reads
+    constexpr int NG = WV ? (F32 ? 4 : 8) : (NW < 4 ? NW : 4);
+    static_assert(NG <= NW, "a vector read covers at most one row vector");
     constexpr int kTeamThreads = TEAM * kWarp;
     __shared__ Moments red[TEAM];
     grid_dependency_wait();
@@ -82,7 +96,7 @@ gated_residual_adaln_kernel(const FusedParams p)
 #pragma unroll
                 for (int h = 0; h < NW / NG; ++h) {
                     f32x2 g[NG];
-                    vec_pairs<F32, NG>(p.gate, goff + EPV * j + 2 * NG * h, g);
+                    seq_pairs<F32, NG, WV>(p.gate, goff + EPV * j + 2 * NG * h, g);
 #pragma unroll
                     for (int e = 0; e < NG; ++e)
                         rv[i][NG * h + e] = f2_to_bf16x2(
@@ -140,8 +154,8 @@ gated_residual_adaln_kernel(const FusedParams p)
 #pragma unroll
             for (int h = 0; h < NW / NG; ++h) {
                 f32x2 hv[NG], cv[NG];
-                vec_pairs<F32, NG>(p.shift, moff + EPV * j + 2 * NG * h, hv);
-                vec_pairs<F32, NG>(p.scale, moff + EPV * j + 2 * NG * h, cv);
+                seq_pairs<F32, NG, WV>(p.shift, moff + EPV * j + 2 * NG * h, hv);
+                seq_pairs<F32, NG, WV>(p.scale, moff + EPV * j + 2 * NG * h, cv);
 #pragma unroll
                 for (int e = 0; e < NG; ++e) {
                     const f32x2 t = f2_fma(f2_from_bf16x2(rv[i][NG * h + e]), r2, b2);
@@ -153,41 +167,41 @@ gated_residual_adaln_kernel(const FusedParams p)
     }
 }
 
-template <int VPT, int NW, int TEAM, bool F32>
+template <int VPT, int NW, int TEAM, bool F32, bool WV>
 cudaError_t launch_one(const FusedParams& p, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)p.pk.num_rows_padded;  // one row per CTA
-    return launch_kernel(gated_residual_adaln_kernel<VPT, NW, TEAM, F32>, grid, TEAM * kWarp, 0, stream, p);
+    return launch_kernel(gated_residual_adaln_kernel<VPT, NW, TEAM, F32, WV>, grid, TEAM * kWarp, 0, stream, p);
 }
 
 // VPT (1..MAXV) as a template argument.
-template <int NW, int TEAM, bool F32, int MAXV, int V = 1>
+template <int NW, int TEAM, bool F32, bool WV, int MAXV, int V = 1>
 cudaError_t launch_vpt(const FusedParams& p, int vpt, cudaStream_t stream)
 {
     if constexpr (V > MAXV) {
         return cudaErrorInvalidValue;
     } else {
         if (vpt == V)
-            return launch_one<V, NW, TEAM, F32>(p, stream);
-        return launch_vpt<NW, TEAM, F32, MAXV, V + 1>(p, vpt, stream);
+            return launch_one<V, NW, TEAM, F32, WV>(p, stream);
+        return launch_vpt<NW, TEAM, F32, WV, MAXV, V + 1>(p, vpt, stream);
     }
 }
 
 // The smallest team of 1, 2, 4 or 8 warps that holds the row in at most
 // MAXV vectors of NW words per lane (the widest rows: 8 warps, up to 8
 // vectors).
-template <int NW, bool F32, int MAXV>
+template <int NW, bool F32, int MAXV, bool WV = false>
 cudaError_t launch_width(const FusedParams& p, cudaStream_t stream)
 {
     const int nvec = p.hidden / (2 * NW);
     auto vpt_for = [&](int team) { return (nvec + team * kWarp - 1) / (team * kWarp); };
     if (vpt_for(1) <= MAXV)
-        return launch_vpt<NW, 1, F32, MAXV>(p, vpt_for(1), stream);
+        return launch_vpt<NW, 1, F32, WV, MAXV>(p, vpt_for(1), stream);
     if (vpt_for(2) <= MAXV)
-        return launch_vpt<NW, 2, F32, MAXV>(p, vpt_for(2), stream);
+        return launch_vpt<NW, 2, F32, WV, MAXV>(p, vpt_for(2), stream);
     if (vpt_for(4) <= MAXV)
-        return launch_vpt<NW, 4, F32, MAXV>(p, vpt_for(4), stream);
-    return launch_vpt<NW, 8, F32, 8>(p, vpt_for(8), stream);
+        return launch_vpt<NW, 4, F32, WV, MAXV>(p, vpt_for(4), stream);
+    return launch_vpt<NW, 8, F32, WV, 8>(p, vpt_for(8), stream);
 }
 
 }  // namespace
@@ -195,11 +209,18 @@ cudaError_t launch_width(const FusedParams& p, cudaStream_t stream)
 // Access width: bf16 vectors take 32-byte accesses when all four row buffers
 // are 32-byte aligned and hidden and every row stride are multiples of 16
 // elements (each row then starts on a 32-byte boundary), else 16-byte ones;
-// fp32 vectors take 16-byte accesses (teams of at most 5 vectors per lane).
+// fp32 vectors take 16-byte accesses (teams of at most 5 vectors per lane),
+// with the vectors read 32 bytes per lane at a time when every sequence's
+// vectors start on a 32-byte boundary (batched varlen 501.7 -> 456.7 us,
+// long video 255.9 -> 244.8 us: each warp load instruction then covers
+// contiguous memory).
 cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream)
 {
-    if (p.mod_f32)
-        return launch_width<4, true, 5>(p, stream);
+    if (p.mod_f32) {
+        const bool vec32 = aligned32(p.gate) && aligned32(p.shift) && aligned32(p.scale) &&
+                           p.gate_seq_stride % 8 == 0 && p.mod_seq_stride % 8 == 0;
+        return vec32 ? launch_width<4, true, 5, true>(p, stream) : launch_width<4, true, 5>(p, stream);
+    }
     const bool wide = aligned32(p.x) && aligned32(p.y) && aligned32(p.res_out) && aligned32(p.norm_out) &&
                       p.hidden % 16 == 0 && p.x_row_stride % 16 == 0 && p.y_row_stride % 16 == 0 &&
                       p.res_row_stride % 16 == 0 && p.norm_row_stride % 16 == 0;

@@ -148,6 +148,19 @@ struct FramesParams {
 cudaError_t launch_frames_to_u8(const FramesParams& p, cudaStream_t stream);
 cudaError_t launch_qk_rmsnorm_rope(const QkParams& p, int head_dim, int rope_mode, cudaStream_t stream);
 cudaError_t launch_adaln_modulate(const AdalnParams& p, cudaStream_t stream);
+
+// How dit_adaln_modulate lays a row out: 2, 4 or 8 words (8-, 16- or 32-byte
+// accesses) per lane vector, a row per warp (team 1) or per CTA of 2, 4 or 8
+// warps, and whether the per-sequence vectors are read 32 bytes at a time.
+// adaln_shape picks it for a call; launch_adaln_shape runs a given one (every
+// shape computes the same result up to the order of the row statistics).
+struct AdalnShape {
+    int row_words;
+    int team;
+    bool wide_vectors;
+};
+AdalnShape adaln_shape(const AdalnParams& p);
+cudaError_t launch_adaln_shape(const AdalnParams& p, const AdalnShape& shape, cudaStream_t stream);
 cudaError_t launch_gated_residual(const GatedParams& p, cudaStream_t stream);
 cudaError_t launch_swiglu(const SwigluParams& p, cudaStream_t stream);
 cudaError_t launch_gated_residual_adaln(const FusedParams& p, cudaStream_t stream);

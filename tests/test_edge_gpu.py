@@ -193,6 +193,24 @@ def test_adaln_row_alignment(offset):
         assert torch.all(t[:, offset + C:].view(torch.int16) == W.SENTINEL)
 
 
+@pytest.mark.parametrize("width", [8, 64, 504, 512, 520, 1024, 1032, 2048, 5632, 13824])
+def test_swiglu_and_residual_every_width(width):
+    """Every launch shape of SwiGLU and the gated residual: one, two or more
+    vectors per lane, 32-byte accesses (widths that are multiples of 16) and
+    16-byte ones (the others), against the oracle."""
+    w = W.custom("widths", (37, 5, 90), (40, 8, 96), hidden=width, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=width, seed=width + 3)
+    rows = w.valid_rows()
+    inp = W.swiglu_inputs(w)
+    out = P.gpu_swiglu(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_swiglu(w, inp, rows)[rows], f"swiglu {width}")
+    P.assert_untouched(out, inp["out"], P.untouched_rows(w), f"swiglu {width}")
+    inp = W.residual_inputs(w)
+    out = P.gpu_residual(w, inp)
+    P.assert_close(P.gather_rows(out, rows), P.oracle_residual(w, inp, rows)[rows], f"residual {width}")
+    P.assert_untouched(out, inp["out"], P.untouched_rows(w), f"residual {width}")
+
+
 def test_swiglu_extreme_activations():
     w = W.custom("sw", (5,), (8,), hidden=8, num_q_heads=1, num_k_heads=1, head_dim=64, inner=64)
     inp = W.swiglu_inputs(w)

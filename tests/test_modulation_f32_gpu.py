@@ -115,3 +115,36 @@ def test_mixed_dtypes_are_rejected():
         dit.dit_adaln_modulate(x, g16, g32, cs, cp)
     with pytest.raises(TypeError):
         dit.dit_gated_residual_adaln(x, x, g32, g16, g16, cs, cp)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("hidden", [2048, 5120])
+def test_vectors_off_a_32_byte_boundary(dtype, hidden):
+    """Per-sequence vectors are read 32 bytes per lane at a time only when
+    every sequence's vectors start on a 32-byte boundary; vectors 16 bytes
+    off one (a legal layout) take the 16-byte reads and give the same
+    results against the oracle, for adaLN and the fused op."""
+    w = W.custom("offvec", (300, 77), (304, 80), hidden=hidden, num_q_heads=1, num_k_heads=1, head_dim=64,
+                 inner=8, seed=hidden + 5)
+    rows = w.valid_rows()
+    inp = W.residual_inputs(w)
+    mod = inp["mod"].to(dtype)
+    per = 16 // mod.element_size()                  # elements in 16 bytes
+    wide = torch.zeros(w.num_seqs, 6 * hidden + 2 * per, dtype=dtype)
+    wide[:, per:per + 6 * hidden] = mod.reshape(w.num_seqs, -1)
+    shifted = wide.cuda()[:, per:per + 6 * hidden].view(w.num_seqs, 6, hidden)   # 16 bytes past the start
+    assert shifted.data_ptr() % 32 == 16
+    cs, cp, _ = P.device_packing(w)
+    x, y = W.rows_view(inp["x"].cuda()), W.rows_view(inp["y"].cuda())
+    ref_inp = dict(inp, mod=mod)
+    out = W.sentinel_like(inp["out"].shape).cuda()
+    dit.dit_adaln_modulate(x, shifted[:, 0], shifted[:, 1], cs, cp, out=W.rows_view(out), eps=w.eps)
+    a_ref = P.oracle_adaln(w, dict(ref_inp, x=inp["x"]), rows)
+    P.assert_close(P.gather_rows(out, rows), a_ref[rows], f"adaln {dtype} off 32 B")
+    res = W.sentinel_like(inp["out"].shape).cuda()
+    norm = W.sentinel_like(inp["out"].shape).cuda()
+    dit.dit_gated_residual_adaln(x, y, shifted[:, 2], shifted[:, 3], shifted[:, 4], cs, cp,
+                                 res_out=W.rows_view(res), norm_out=W.rows_view(norm), eps=w.eps)
+    r_ref, n_ref = P.oracle_fused(w, ref_inp, rows)
+    P.assert_close(P.gather_rows(res, rows), r_ref[rows], f"fused residual {dtype} off 32 B")
+    P.assert_close(P.gather_rows(norm, rows), n_ref[rows], f"fused norm {dtype} off 32 B")
