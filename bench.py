@@ -1096,6 +1096,54 @@ def run_host_overhead(args):
         print(f"| {name} | {(t1 - t0) / n * 1e6:.2f} | {(t3 - t2) / n * 1e6:.2f} |", flush=True)
 
 
+def run_profile_op(args):
+    """One operator alone, at the workload's full shape, with only its own
+    buffers on the device (adaLN on batched varlen: 2 x 718 MB): W + K
+    launches back to back, then a synchronize.  For a profiler capture of a
+    single full-size launch (e.g. ncu -k regex:adaln_ -s W -c 1)."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from dit_token_b200 import build
+    build.build()
+    w = W.workload(args.workload, args.seed)
+    op = args.profile_op
+    builders = {"qk_rmsnorm_rope": lambda: {"qk": W.qk_inputs(w)},
+                "adaln_modulate": lambda: {"adaln": W.adaln_inputs(w)},
+                "gated_residual": lambda: {"res": W.residual_inputs(w)},
+                "swiglu": lambda: {"swiglu": W.swiglu_inputs(w)}}
+    host = builders[op]()
+
+    class OneOp(Step):
+        def __init__(self):
+            import dit_token_b200 as dit
+            self.dit, self.w = dit, w
+            self.cs = torch.from_numpy(w.cu_seqlens).to(device)
+            self.cp = torch.from_numpy(w.cu_seqlens_padded).to(device)
+            self.grid = None if w.rope_grid is None else torch.from_numpy(w.rope_grid).to(device)
+            self.pos_offset = None if w.pos_offset is None else torch.from_numpy(w.pos_offsets).to(device)
+            rv = W.rows_view
+            self.v = {}
+            if "qk" in host:
+                self.q, self.k = host["qk"]["q"].to(device), host["qk"]["k"].to(device)
+                self.wq, self.wk = host["qk"]["q_weight"].to(device), host["qk"]["k_weight"].to(device)
+                self.v.update(q=rv(self.q), k=rv(self.k))
+            if "adaln" in host:
+                ax, ao, mod = (host["adaln"][k].to(device) for k in ("x", "out", "mod"))
+                self.v.update(ax=rv(ax), aout=rv(ao), shift=mod[:, 0], scale=mod[:, 1])
+            if "res" in host:
+                rx, ry, ro, mod = (host["res"][k].to(device) for k in ("x", "y", "out", "mod"))
+                self.v.update(rx=rv(rx), ry=rv(ry), rout=rv(ro), gate=mod[:, 2])
+            if "swiglu" in host:
+                ab, so = host["swiglu"]["ab"].to(device), host["swiglu"]["out"].to(device)
+                self.v.update(a=rv(ab)[:, : w.inner], b=rv(ab)[:, w.inner:], sout=rv(so))
+
+    one = OneOp()
+    for _ in range(args.warmup + args.steps):
+        one.run_op(op)
+    torch.cuda.synchronize(device)
+    print(f"{op} on {w.name}: {args.warmup + args.steps} launches", flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -1121,6 +1169,9 @@ def main(argv=None):
                     help="print a markdown table of the operator variants instead of the JSON line")
     ap.add_argument("--host-overhead", action="store_true",
                     help="print the host time per call of every entry point (tiny workload, no sync)")
+    ap.add_argument("--profile-op", choices=OPS,
+                    help="launch only this operator, W + K times on the workload with its own buffers "
+                         "(for a profiler capture of one full-size launch)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -1128,7 +1179,9 @@ def main(argv=None):
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
-    if args.host_overhead:
+    if args.profile_op:
+        run_profile_op(args)
+    elif args.host_overhead:
         run_host_overhead(args)
     elif args.table:
         run_table(args)

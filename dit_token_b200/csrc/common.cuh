@@ -9,7 +9,6 @@ namespace dit {
 
 constexpr int kWarp = 32;
 constexpr int kCtaThreads = 256;          // 8 warps
-constexpr int kWarpsPerCta = kCtaThreads / kWarp;
 
 // ---------------------------------------------- dependent launches
 // Called first in every kernel, before any global-memory access: waits until
@@ -85,40 +84,6 @@ __device__ __forceinline__ bool map_valid_row(int v, const int32_t* __restrict__
     s.local = r;
     return true;
 }
-
-// Walks valid-row ordinals upward for a persistent CTA that owns a contiguous
-// range of them: the padded row of the next ordinal is the previous one + 1
-// except at a sequence boundary, so global loads happen only when a boundary
-// is crossed.  Every thread of the CTA holds the same state.
-struct RowCursor {
-    const int32_t* cs;
-    const int32_t* cp;
-    int B;
-    int rows_padded;
-    int b;  // current sequence
-    int cs0, cs1, cp0, cp1;
-
-    __device__ __forceinline__ void load(int bb)
-    {
-        b = bb;
-        cs0 = __ldg(cs + b);
-        cs1 = __ldg(cs + b + 1);
-        cp0 = __ldg(cp + b);
-        cp1 = __ldg(cp + b + 1);
-    }
-    // Padded row of ordinal v (v never decreases between calls), or -1 when v
-    // is not a valid row or the descriptor points outside the buffer.
-    __device__ __forceinline__ int row(int v)
-    {
-        while (v >= cs1 && b + 1 < B)
-            load(b + 1);
-        const int r = v - cs0;
-        if (r < 0 || r >= cs1 - cs0 || r >= cp1 - cp0)
-            return -1;
-        const long long rr = (long long)cp0 + r;
-        return rr < rows_padded ? (int)rr : -1;
-    }
-};
 
 // ---------------------------------------------------------- vector I/O
 // Streamed activations are touched once: load and store them with the
@@ -209,12 +174,6 @@ __device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
 typedef float2 f32x2;
 
 __device__ __forceinline__ f32x2 f2_make(float lo, float hi) { return make_float2(lo, hi); }
-
-__device__ __forceinline__ void f2_split(f32x2 v, float& lo, float& hi)
-{
-    lo = v.x;
-    hi = v.y;
-}
 
 // bf16x2 word (element 0 in the low half) -> the two values as an fp32 pair.
 __device__ __forceinline__ f32x2 f2_from_bf16x2(uint32_t w)
@@ -351,28 +310,6 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8])
 {
     return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
-
-// Barrier among the TEAM warps of team `team` only (hardware named barrier
-// 1 + team; id 0 stays __syncthreads'), so the row teams of one CTA never
-// wait for each other.
-template <int TEAM>
-__device__ __forceinline__ void team_barrier(int team)
-{
-    if (TEAM == kWarpsPerCta)
-        __syncthreads();
-    else
-        asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "n"(TEAM * kWarp) : "memory");
-}
-
-// Minimum resident CTAs per SM to ask of a row kernel holding VPT 16-byte
-// vectors per lane of each of INPUTS streamed inputs at once (about
-// 4 * INPUTS * VPT + EXTRA registers per thread).
-template <int VPT, int INPUTS = 1, int EXTRA = 28>
-struct MinCtas {
-    static constexpr int regs = 4 * INPUTS * VPT + EXTRA;
-    static constexpr int raw = 65536 / (kCtaThreads * regs);
-    static constexpr int value = raw < 1 ? 1 : (raw > 8 ? 8 : raw);
-};
 
 // ----------------------------------------------- row mean / variance
 // LayerNorm statistics in one pass, robust to large means and outliers: each

@@ -141,3 +141,62 @@ def test_dependent_chain_equals_synchronized_run(chain, graphed):
             for name, t in (("r", d["r"]), ("s", d["s"]), ("q", d["a"]), ("k", d["k"])):
                 assert torch.equal(t.view(torch.int16), ref[name].view(torch.int16)), f"round {i} {name}"
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("graphed", [False, True])
+def test_descriptor_written_by_the_previous_kernel(graphed):
+    """A kernel's first reads are the packing descriptors, which the
+    previous kernel on the stream may have just written: dit_av_stream_seqlens
+    writes the per-stream descriptor into buffers that are reset every round
+    (to an empty descriptor, which would make adaLN write nothing) and the
+    per-stream adaLN reads it right away.  Twelve rounds back to back, eagerly
+    and as a replayed graph; the outputs equal the synchronized run's bit for
+    bit, and the oracle's per-stream adaLN."""
+    w = W.custom("desc", (6100, 900, 3000), (6144, 1024, 3072), hidden=2048, num_q_heads=1, num_k_heads=1,
+                 head_dim=64, inner=8, grids=((5, 24, 42), (0, 0, 0), (2, 24, 42)), seed=91)
+    C, B = w.hidden, w.num_seqs
+    rows = w.valid_rows()
+    cs, cp, grid = P.device_packing(w)
+    m = W.modulation_av(w)
+    mv = m.cuda().view(2 * B, 6, C)
+    inp = W.adaln_inputs(w)
+    x = W.rows_view(inp["x"].cuda())
+    out = W.sentinel_like(inp["out"].shape).cuda()
+    cs2 = torch.zeros(2 * B + 1, dtype=torch.int32, device="cuda")
+    cp2 = torch.zeros_like(cs2)
+    sentinel = W.sentinel_like(inp["out"].shape).cuda()
+
+    def one_round(sync=False):
+        out.copy_(sentinel)
+        cs2.zero_()
+        cp2.zero_()
+        dit.dit_av_stream_seqlens(cs, cp, grid, out=(cs2, cp2))
+        if sync:
+            torch.cuda.synchronize()
+        dit.dit_adaln_modulate(x, mv[:, 0], mv[:, 1], cs2, cp2, out=W.rows_view(out), eps=w.eps)
+        if sync:
+            torch.cuda.synchronize()
+
+    one_round(sync=True)
+    ref = out.clone()
+    import oracle
+    flat = P.mod_flat(m)
+    o = oracle.adaln_modulate(tbits(W.rows_view(inp["x"])), flat, flat[C:], w.cu_seqlens, w.cu_seqlens_padded,
+                              hidden=C, eps=w.eps, mod_seq_stride=12 * C, audio_offset=6 * C, rows=rows,
+                              rope_grid=w.rope_grid)
+    P.assert_close(P.gather_rows(ref, rows), o[rows], "per-stream adaln, synchronized")
+    run = one_round
+    if graphed:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            one_round()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one_round()
+        run = g.replay
+    for i in range(12):
+        run()
+        # (the comparison synchronizes between rounds, never inside one)
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"round {i}"
