@@ -35,16 +35,16 @@ namespace {
 constexpr int kRowWarps = 4;                 // rows (warps) per CTA of the warp-per-row kernel
 constexpr int kRowCtaThreads = kRowWarps * kWarp;
 
-// Statistics of the VPT vectors of NW words a lane holds (vectors at or past
-// nvec are empty), merged over the warp.  Vector i of the lane is vector
-// i * STRIDE + lane_vec0 of the row.
+// Statistics of the warp's share of a row: the VPT vectors of NW words each
+// lane holds (vectors at or past nvec are empty), about lane 0's first
+// element.  Vector i of the lane is vector i * STRIDE + lane_vec0 of the row.
 template <int VPT, int NW, int STRIDE>
 __device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW], int lane_vec0, int nvec)
 {
-    const float k = bf16_lo(xv[0][0]);
+    const int lane = threadIdx.x & (kWarp - 1);
+    const float k = __shfl_sync(0xffffffffu, bf16_lo(xv[0][0]), 0);
     const f32x2 kk = f2_make(k, k);
     f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
-    float cnt = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         if (i * STRIDE + lane_vec0 < nvec) {
@@ -54,10 +54,10 @@ __device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW
                 s2 = f2_add(s2, d);
                 q2 = f2_fma(d, d, q2);
             }
-            cnt += (float)(2 * NW);
         }
     }
-    return moments_warp(moments_from_sums(cnt, k, s2.x + s2.y, q2.x + q2.y));
+    const int nv = warp_vector_count<VPT, STRIDE>(lane_vec0 - lane, nvec);
+    return warp_moments((float)(2 * NW * nv), k, s2, q2);
 }
 
 // 2 * NP output elements (NP words): (x * rstd + nb) * (1 + scale) + shift,

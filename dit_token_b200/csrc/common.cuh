@@ -312,12 +312,15 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8])
 }
 
 // ----------------------------------------------- row mean / variance
-// LayerNorm statistics in one pass, robust to large means and outliers: each
-// thread accumulates s = sum(x - k) and q = sum((x - k)^2) about its own first
-// value k, turns them into (count, mean, M2 = sum of squared deviations), and
-// the partial moments are merged pairwise (Chan, Golub and LeVeque's update):
+// LayerNorm statistics in one pass, robust to large means and outliers: the
+// lanes of a warp accumulate s = sum(x - k) and q = sum((x - k)^2) about one
+// shift k common to the warp (a value of the row: lane 0's first element), the
+// sums are added over the warp, and become (count, mean, M2 = sum of squared
+// deviations).  Warps that share a row merge their moments pairwise (Chan,
+// Golub and LeVeque's update):
 //   n = na + nb,  d = mb - ma,  mean = ma + d nb / n,  M2 = Ma + Mb + d^2 na nb / n.
-// The merge order is fixed, so the result is bitwise reproducible.
+// The summation and merge orders are fixed, so the result is bitwise
+// reproducible.
 struct Moments {
     float n, mean, m2;
 };
@@ -340,17 +343,29 @@ __device__ __forceinline__ Moments moments_from_sums(float n, float k, float s, 
     return Moments{n, k + m, fmaxf(q - s * m, 0.f)};
 }
 
-// Merge over the 32 lanes of a warp (xor butterfly: every lane ends with the total).
-__device__ __forceinline__ Moments moments_warp(Moments m)
+// Moments of a warp's n values from each lane's sums s2 (of x - k) and q2 (of
+// (x - k)^2), kept as fp32 pairs, about the warp's common shift k: the sums
+// are added over the 32 lanes by an xor butterfly (both lanes of a pair add
+// the same two operands, so every lane ends with the same totals).
+__device__ __forceinline__ Moments warp_moments(float n, float k, f32x2 s2, f32x2 q2)
 {
+    f32x2 sq = f2_make(s2.x + s2.y, q2.x + q2.y);
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        Moments other{__shfl_xor_sync(0xffffffffu, m.n, o), __shfl_xor_sync(0xffffffffu, m.mean, o),
-                      __shfl_xor_sync(0xffffffffu, m.m2, o)};
-        // lanes of a pair merge in the same (lower lane first) order
-        m = (threadIdx.x & o) ? moments_merge(other, m) : moments_merge(m, other);
-    }
-    return m;
+    for (int o = 16; o >= 1; o >>= 1)
+        sq = f2_add(sq, f2_make(__shfl_xor_sync(0xffffffffu, sq.x, o), __shfl_xor_sync(0xffffffffu, sq.y, o)));
+    return moments_from_sums(n, k, sq.x, sq.y);
+}
+
+// How many of the vectors i * STRIDE + warp_vec0 + lane (i < VPT, lane < 32)
+// fall below nvec: the vectors a warp holds of a row.
+template <int VPT, int STRIDE>
+__device__ __forceinline__ int warp_vector_count(int warp_vec0, int nvec)
+{
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+        n += min(max(nvec - (i * STRIDE + warp_vec0), 0), kWarp);
+    return n;
 }
 
 template <int WIDTH>

@@ -111,11 +111,11 @@ gated_residual_adaln_kernel(const FusedParams p)
         }
     }
 
-    // LN statistics of the stored residual: shifted sums, merged as moments
-    const float k = bf16_lo(rv[0][0]);
+    // LN statistics of the stored residual: sums about lane 0's first value,
+    // added over the warp, merged across the team as moments
+    const float k = __shfl_sync(0xffffffffu, bf16_lo(rv[0][0]), 0);
     const f32x2 kk = f2_make(k, k);
     f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
-    float cnt = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         if (i * kTeamThreads + tt < nvec) {
@@ -125,10 +125,10 @@ gated_residual_adaln_kernel(const FusedParams p)
                 s2 = f2_add(s2, d);
                 q2 = f2_fma(d, d, q2);
             }
-            cnt += (float)EPV;
         }
     }
-    Moments m = moments_warp(moments_from_sums(cnt, k, s2.x + s2.y, q2.x + q2.y));
+    const int nv = warp_vector_count<VPT, kTeamThreads>(tt - lane, nvec);
+    Moments m = warp_moments((float)(EPV * nv), k, s2, q2);
     if (TEAM > 1) {
         if (lane == 0)
             red[warp] = m;
