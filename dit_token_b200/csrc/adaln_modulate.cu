@@ -8,9 +8,10 @@
 // team of 2-8 warps for wide rows, in short-lived CTAs, so the hardware keeps
 // every SM filled with new rows as old ones finish.  A lane holds VPT vectors
 // of 4, 8 or 16 elements (8-, 16- or 32-byte accesses).  Statistics in one
-// pass: per-lane sums about the lane's first value, merged as (count, mean,
-// M2) moments by warp shuffles (and across a team through shared memory,
-// behind one barrier).  Output pass: per element (x * rstd - mean * rstd) *
+// pass: per-lane sums of x - k and (x - k)^2 about one value k of the warp
+// (lane 0's first element), added over the warp by shuffles and turned into
+// (count, mean, M2) moments, which a team merges through shared memory
+// behind one barrier.  Output pass: per element (x * rstd - mean * rstd) *
 // (1 + scale) + shift in packed fp32 pairs, the per-sequence vectors read
 // through the read-only path (they stay in L1/L2: every row of a sequence
 // reads the same 2 * hidden values), 16 or 32 bytes per lane at a time.  HBM
@@ -34,31 +35,6 @@ namespace {
 
 constexpr int kRowWarps = 4;                 // rows (warps) per CTA of the warp-per-row kernel
 constexpr int kRowCtaThreads = kRowWarps * kWarp;
-
-// Statistics of the warp's share of a row: the VPT vectors of NW words each
-// lane holds (vectors at or past nvec are empty), about lane 0's first
-// element.  Vector i of the lane is vector i * STRIDE + lane_vec0 of the row.
-template <int VPT, int NW, int STRIDE>
-__device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW], int lane_vec0, int nvec)
-{
-    const int lane = threadIdx.x & (kWarp - 1);
-    const float k = __shfl_sync(0xffffffffu, bf16_lo(xv[0][0]), 0);
-    const f32x2 kk = f2_make(k, k);
-    f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        if (i * STRIDE + lane_vec0 < nvec) {
-#pragma unroll
-            for (int e = 0; e < NW; ++e) {
-                const f32x2 d = f2_sub(f2_from_bf16x2(xv[i][e]), kk);
-                s2 = f2_add(s2, d);
-                q2 = f2_fma(d, d, q2);
-            }
-        }
-    }
-    const int nv = warp_vector_count<VPT, STRIDE>(lane_vec0 - lane, nvec);
-    return warp_moments((float)(2 * NW * nv), k, s2, q2);
-}
 
 // 2 * NP output elements (NP words): (x * rstd + nb) * (1 + scale) + shift,
 // with the sequence's vectors read at element `moff_elem`: 32 bytes at a time
@@ -143,7 +119,7 @@ adaln_row_kernel(const AdalnParams p)
     const int nvec = p.hidden / (2 * NW);
     uint32_t xv[VPT][NW];
     load_row<VPT, NW, kWarp>(p.x + (int64_t)s.row * p.x_row_stride, lane, nvec, xv);
-    const Moments m = lane_row_moments<VPT, NW, kWarp>(xv, lane, nvec);
+    const Moments m = row_moments<VPT, NW, 1>(xv, nvec, nullptr, nullptr, nullptr);
     const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);
     modulate_row<VPT, NW, kWarp, F32, WV>(xv, lane, nvec, rstd, m.mean, p, s);
 }
@@ -156,10 +132,10 @@ __global__ void __launch_bounds__(TEAM * kWarp)
 adaln_team_kernel(const AdalnParams p)
 {
     constexpr int kTeamThreads = TEAM * kWarp;
-    __shared__ Moments red[TEAM];
+    __shared__ Moments red[TEAM], red2[TEAM];
+    __shared__ int far_w[TEAM];
     grid_dependency_wait();
     const int lane = threadIdx.x & (kWarp - 1);
-    const int warp = threadIdx.x >> 5;
     const int tt = threadIdx.x;
     RowSlot s;
     if (!map_valid_row(blockIdx.x, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded,
@@ -168,14 +144,7 @@ adaln_team_kernel(const AdalnParams p)
     const int nvec = p.hidden / (2 * NW);
     uint32_t xv[VPT][NW];
     load_row<VPT, NW, kTeamThreads>(p.x + (int64_t)s.row * p.x_row_stride, tt, nvec, xv);
-    Moments m = lane_row_moments<VPT, NW, kTeamThreads>(xv, tt, nvec);
-    if (lane == 0)
-        red[warp] = m;
-    __syncthreads();
-    m = red[0];
-#pragma unroll
-    for (int w = 1; w < TEAM; ++w)
-        m = moments_merge(m, red[w]);
+    const Moments m = row_moments<VPT, NW, TEAM>(xv, nvec, red, red2, far_w);
     const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);
     modulate_row<VPT, NW, kTeamThreads, F32, WV>(xv, tt, nvec, rstd, m.mean, p, s);
 }

@@ -347,13 +347,20 @@ __device__ __forceinline__ Moments moments_from_sums(float n, float k, float s, 
 // (x - k)^2), kept as fp32 pairs, about the warp's common shift k: the sums
 // are added over the 32 lanes by an xor butterfly (both lanes of a pair add
 // the same two operands, so every lane ends with the same totals).
-__device__ __forceinline__ Moments warp_moments(float n, float k, f32x2 s2, f32x2 q2)
+// M2 = q - s^2 / n (and the mean, k + s / n) cancel when k lies far from the
+// mean -- a massive activation in the channel k is taken from: `far` reports
+// a shift more than 4 standard deviations away (s^2 / n > 16 M2), where up to
+// 4 of fp32's 24 bits are lost; the caller then sums the row again about the
+// mean just found (within a small fraction of a deviation of the true one).
+__device__ __forceinline__ Moments warp_moments(float n, float k, f32x2 s2, f32x2 q2, bool& far)
 {
     f32x2 sq = f2_make(s2.x + s2.y, q2.x + q2.y);
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1)
         sq = f2_add(sq, f2_make(__shfl_xor_sync(0xffffffffu, sq.x, o), __shfl_xor_sync(0xffffffffu, sq.y, o)));
-    return moments_from_sums(n, k, sq.x, sq.y);
+    const Moments m = moments_from_sums(n, k, sq.x, sq.y);
+    far = sq.x * (m.mean - k) > 16.f * m.m2;
+    return m;
 }
 
 // How many of the vectors i * STRIDE + warp_vec0 + lane (i < VPT, lane < 32)
@@ -366,6 +373,79 @@ __device__ __forceinline__ int warp_vector_count(int warp_vec0, int nvec)
     for (int i = 0; i < VPT; ++i)
         n += min(max(nvec - (i * STRIDE + warp_vec0), 0), kWarp);
     return n;
+}
+
+// Statistics of the warp's share of a row: the VPT vectors of NW words each
+// lane holds (vectors at or past nvec are empty), about the shift k (common
+// to the warp).  Vector i of the lane is vector i * STRIDE + lane_vec0 of the
+// row.
+template <int VPT, int NW, int STRIDE>
+__device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW], int lane_vec0, int nvec,
+                                                    float k, bool& far)
+{
+    const int lane = threadIdx.x & (kWarp - 1);
+    const f32x2 kk = f2_make(k, k);
+    f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        if (i * STRIDE + lane_vec0 < nvec) {
+#pragma unroll
+            for (int e = 0; e < NW; ++e) {
+                const f32x2 d = f2_sub(f2_from_bf16x2(xv[i][e]), kk);
+                s2 = f2_add(s2, d);
+                q2 = f2_fma(d, d, q2);
+            }
+        }
+    }
+    const int nv = warp_vector_count<VPT, STRIDE>(lane_vec0 - lane, nvec);
+    return warp_moments((float)(2 * NW * nv), k, s2, q2, far);
+}
+
+// The row's moments: sums about lane 0's first element of each warp, merged
+// across a team of TEAM warps (TEAM > 1: through shared memory, behind a
+// barrier); summed again about the mean found when a warp's shift lay far
+// from it.  red, red2 and far_w: TEAM entries of shared memory.
+template <int VPT, int NW, int TEAM>
+__device__ __forceinline__ Moments row_moments(const uint32_t (&xv)[VPT][NW], int nvec, Moments* red,
+                                               Moments* red2, int* far_w)
+{
+    constexpr int STRIDE = TEAM * kWarp;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int warp = threadIdx.x >> 5;
+    // the lane's first vector: a warp per row (several rows per CTA) or a
+    // team per row (one row per CTA)
+    const int tt = TEAM == 1 ? lane : (int)threadIdx.x;
+    bool far;
+    Moments m = lane_row_moments<VPT, NW, STRIDE>(xv, tt, nvec, __shfl_sync(0xffffffffu, bf16_lo(xv[0][0]), 0),
+                                                  far);
+    if constexpr (TEAM > 1) {
+        if (lane == 0) {
+            red[warp] = m;
+            far_w[warp] = far;
+        }
+        __syncthreads();
+        m = red[0];
+        far = far_w[0] != 0;
+#pragma unroll
+        for (int w = 1; w < TEAM; ++w) {
+            m = moments_merge(m, red[w]);
+            far = far || far_w[w] != 0;
+        }
+    }
+    if (far) {  // uniform over the warp (TEAM 1) or the CTA
+        bool unused;
+        m = lane_row_moments<VPT, NW, STRIDE>(xv, tt, nvec, m.mean, unused);
+        if constexpr (TEAM > 1) {
+            if (lane == 0)
+                red2[warp] = m;
+            __syncthreads();
+            m = red2[0];
+#pragma unroll
+            for (int w = 1; w < TEAM; ++w)
+                m = moments_merge(m, red2[w]);
+        }
+    }
+    return m;
 }
 
 template <int WIDTH>

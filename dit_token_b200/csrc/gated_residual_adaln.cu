@@ -57,11 +57,11 @@ gated_residual_adaln_kernel(const FusedParams p)
     constexpr int NG = WV ? (F32 ? 4 : 8) : (NW < 4 ? NW : 4);
     static_assert(NG <= NW, "a vector read covers at most one row vector");
     constexpr int kTeamThreads = TEAM * kWarp;
-    __shared__ Moments red[TEAM];
+    __shared__ Moments red[TEAM], red2[TEAM];
+    __shared__ int far_w[TEAM];
     grid_dependency_wait();
 
     const int lane = threadIdx.x & (kWarp - 1);
-    const int warp = threadIdx.x >> 5;
     const int tt = threadIdx.x;
     RowSlot s;
     if (!map_valid_row(blockIdx.x, p.pk.cu_seqlens, p.pk.cu_seqlens_padded, p.pk.num_seqs, p.pk.num_rows_padded,
@@ -111,33 +111,8 @@ gated_residual_adaln_kernel(const FusedParams p)
         }
     }
 
-    // LN statistics of the stored residual: sums about lane 0's first value,
-    // added over the warp, merged across the team as moments
-    const float k = __shfl_sync(0xffffffffu, bf16_lo(rv[0][0]), 0);
-    const f32x2 kk = f2_make(k, k);
-    f32x2 s2 = f2_make(0.f, 0.f), q2 = f2_make(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        if (i * kTeamThreads + tt < nvec) {
-#pragma unroll
-            for (int e = 0; e < NW; ++e) {
-                const f32x2 d = f2_sub(f2_from_bf16x2(rv[i][e]), kk);
-                s2 = f2_add(s2, d);
-                q2 = f2_fma(d, d, q2);
-            }
-        }
-    }
-    const int nv = warp_vector_count<VPT, kTeamThreads>(tt - lane, nvec);
-    Moments m = warp_moments((float)(EPV * nv), k, s2, q2);
-    if (TEAM > 1) {
-        if (lane == 0)
-            red[warp] = m;
-        __syncthreads();
-        m = red[0];
-#pragma unroll
-        for (int w = 1; w < TEAM; ++w)
-            m = moments_merge(m, red[w]);
-    }
+    // LN statistics of the stored residual (as adaLN's)
+    const Moments m = row_moments<VPT, NW, TEAM>(rv, nvec, red, red2, far_w);
     const float rstd = rsqrtf(m.m2 * (1.0f / (float)p.hidden) + p.eps);  // as in adaln_modulate.cu
     const f32x2 r2 = f2_make(rstd, rstd);
     const float nb = -m.mean * rstd;
