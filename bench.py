@@ -238,6 +238,17 @@ class ClockSampler:
                 "window_s": round(t1 - t0, 4), "source": self.source}
 
 
+def clock_note(sampler: ClockSampler) -> str:
+    """One line on the SM clock over a whole --table / --variants run."""
+    sampler.stop()
+    c = sampler.summary(float("-inf"), float("inf"))
+    if not c["samples"]:
+        return "\nSM clock: not sampled (no NVML or nvidia-smi)"
+    return (f"\nSM clock over the run: median {c['sm_mhz']:.0f} MHz (min {c['sm_mhz_min']:.0f}, max "
+            f"{c['sm_mhz_max']:.0f}; clocks.max.sm {c['sm_max_mhz']:.0f}), reasons {c['reasons'] or 'none'}, "
+            f"peak power {c['power_w_max']} W, {c['samples']} samples ({c['source']})")
+
+
 def spread(values_ms) -> dict:
     """Median, 10th and 90th percentile of per-step (or per-launch) times, in us."""
     v = np.asarray(list(values_ms), dtype=np.float64) * 1e3
@@ -881,6 +892,8 @@ def run_table(args):
         torch.cuda.synchronize(device)
         return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3  # us
 
+    sampler = ClockSampler(0)
+    sampler.start()
     print(f"| workload | op | GPU us | tokens/s | GB/s | % of 8 TB/s | % of {kind} {peak:.0f} GB/s |")
     print("|---|---|---|---|---|---|---|")
     for name in W.WORKLOAD_NAMES:
@@ -907,6 +920,7 @@ def run_table(args):
     gbs = 5 * FRAMES_ELEMS / (us * 1e-6) / 1e9
     print(f"| frames 1x3x243x768x1344 | frames_to_u8 (BTHWC) | {us:.1f} | - | {gbs:.0f} | "
           f"{100 * gbs / 8000:.1f} | {100 * gbs / peak:.1f} |", flush=True)
+    print(clock_note(sampler), flush=True)
 
 
 def run_variants(args):
@@ -942,6 +956,8 @@ def run_variants(args):
         print(f"| {wname} | {op} | {variant} | {us:.1f} | {tokens / (us * 1e-6):.3g} | {gbs:.0f} | "
               f"{100 * gbs / peak:.1f} |", flush=True)
 
+    sampler = ClockSampler(0)
+    sampler.start()
     print(f"| workload | op | variant | GPU us | tokens/s | GB/s | % of {kind} {peak:.0f} GB/s |")
     print("|---|---|---|---|---|---|---|")
     for name in ("batched_varlen", "long_video"):
@@ -1006,6 +1022,7 @@ def run_variants(args):
         ab[:, :512], ab[:, 512:], cs, cs, out=out)), 6 * 512 * n, n)
     del ab, out
     torch.cuda.empty_cache()
+    print(clock_note(sampler), flush=True)
 
 
 def run_host_overhead(args):
