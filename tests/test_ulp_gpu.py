@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import dit_token_b200 as dit
 from dit_token_b200 import workloads as W
 import _parity as P
 
@@ -138,3 +139,50 @@ def test_adaln_statistics_on_hard_rows(hidden):
     r_ref, n_ref = P.oracle_fused(w, inp, rows)
     assert np.array_equal(P.gather_rows(res, rows), r_ref[rows])
     check_hard(f"fused {hidden}", P.gather_rows(norm, rows), n_ref[rows], n)
+
+
+@pytest.mark.parametrize("hidden", [3072, 5120])
+@pytest.mark.parametrize("layout", ["rows on a 16-byte boundary", "fp32 vectors"])
+def test_adaln_statistics_on_hard_rows_other_layouts(hidden, layout):
+    """The same rows through the kernels' other instantiations: 16-byte row
+    accesses (rows starting 8 elements into a wider buffer, so not on a
+    32-byte boundary) and fp32 modulation vectors."""
+    n = 24
+    nrows = n * len(HARD_KINDS)
+    w = W.custom("hard", (nrows // 2, nrows // 2), (nrows // 2 + 4, nrows // 2 + 4), hidden=hidden,
+                 num_q_heads=1, num_k_heads=1, head_dim=64, inner=8, seed=hidden + 1)
+    rows = w.valid_rows()
+    x = hard_rows(n, hidden, seed=hidden + 1)
+    inp = W.adaln_inputs(w)
+    res_inp = W.residual_inputs(w)
+    for d in (inp, res_inp):
+        W.rows_view(d["x"])[torch.from_numpy(rows)] = x
+    res_inp["y"].zero_()
+    if layout == "fp32 vectors":
+        inp["mod"] = W.modulation(w, torch.float32)
+        res_inp["mod"] = inp["mod"]
+        out = P.gpu_adaln(w, inp)
+        res, norm = P.gpu_fused(w, res_inp)
+        got_a, got_r, got_n = (P.gather_rows(t, rows) for t in (out, res, norm))
+    else:
+        cs, cp, _ = P.device_packing(w)
+        mod = inp["mod"].cuda()
+        C, off = hidden, 8
+
+        def wide(src=None):
+            buf = W.sentinel_like((inp["x"].shape[0], C + 16)).cuda()
+            if src is not None:
+                buf[:, off:off + C] = src.cuda()
+            return buf, W.rows_view(buf)[:, off:off + C]
+
+        (_, xa), (ob, oa) = wide(inp["x"]), wide()
+        dit.dit_adaln_modulate(xa, mod[:, 0], mod[:, 1], cs, cp, out=oa, eps=w.eps)
+        (_, xf), (_, yf), (rb, rf), (nb, nf) = wide(res_inp["x"]), wide(res_inp["y"]), wide(), wide()
+        dit.dit_gated_residual_adaln(xf, yf, mod[:, 2], mod[:, 3], mod[:, 4], cs, cp, res_out=rf, norm_out=nf,
+                                     eps=w.eps)
+        torch.cuda.synchronize()
+        got_a, got_r, got_n = (P.gather_rows(t[:, off:off + C].contiguous(), rows) for t in (ob, rb, nb))
+    check_hard(f"adaln {hidden} {layout}", got_a, P.oracle_adaln(w, inp, rows)[rows], n)
+    r_ref, n_ref = P.oracle_fused(w, res_inp, rows)
+    assert np.array_equal(got_r, r_ref[rows])
+    check_hard(f"fused {hidden} {layout}", got_n, n_ref[rows], n)
