@@ -46,3 +46,32 @@ def test_reference_arm_line():
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_clock_summary_and_note():
+    """The clock record of a run (host logic, canned samples): only samples
+    inside the timed window count when there are any; the reasons are the
+    union of the samples' reasons; the one-line note of --table / --variants
+    reports the median and the reasons."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Canned(bench.ClockSampler):
+        def __init__(self, samples):
+            self.samples, self.max_mhz, self.source = samples, 1965.0, "canned"
+
+        def stop(self):
+            pass
+
+    s = Canned([(0.5, 1965.0, [], 200.0), (1.0, 1800.0, ["sw_power_cap"], 500.0), (2.0, 1700.0, [], 480.0),
+                (9.0, 1000.0, ["hw_slowdown"], 100.0)])
+    c = s.summary(0.9, 2.1)
+    assert c["samples"] == 2 and c["in_timed_window"] is True
+    assert c["sm_mhz"] == 1750.0 and c["sm_mhz_min"] == 1700.0 and c["sm_mhz_max"] == 1800.0
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 500.0
+    outside = s.summary(3.0, 4.0)  # no sample inside: every sample counts, flagged as such
+    assert outside["samples"] == 4 and outside["in_timed_window"] is False
+    assert outside["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    note = bench.clock_note(s)
+    assert "median 1750 MHz" in note and "hw_slowdown" in note and "4 samples" in note
+    assert "not sampled" in bench.clock_note(Canned([]))
