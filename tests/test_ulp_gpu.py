@@ -118,10 +118,11 @@ def check_hard(what, gpu_bits, ref_bits, n_per_kind):
         print(f"{what} {kind}: {share:.5f} bit-identical, max error {err.max():.3g}")
 
 
-@pytest.mark.parametrize("hidden", [2048, 3072, 5120])
+@pytest.mark.parametrize("hidden", [2048, 3072, 5120, 8192, 16384])
 def test_adaln_statistics_on_hard_rows(hidden):
     """adaLN and the fused residual + adaLN on rows built to defeat one-pass
-    statistics; 2048 and 3072 take a warp per row, 5120 a 2-warp team."""
+    statistics; 2048 and 3072 take a warp per row, 5120 and wider a team of
+    warps (2 at 5120 and 8192, 4 at 16384; the fused op's teams are wider)."""
     n = 24
     nrows = n * len(HARD_KINDS)
     w = W.custom("hard", (nrows // 2, nrows // 2), (nrows // 2 + 4, nrows // 2 + 4), hidden=hidden,
