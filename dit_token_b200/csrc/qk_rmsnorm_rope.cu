@@ -9,8 +9,9 @@
 // per-head sum of squares is a log2(LPH)-step xor-shuffle reduction.  A lane
 // always sits at the same place inside a head, so it needs the cos/sin of
 // only its own 4 pairs: it computes them once per row (angle reduced in fp64,
-// then sincosf) and reuses them for all num_q_heads + num_k_heads heads of
-// that row -- cos/sin are never re-read or recomputed per head.  The heads
+// then the hardware sine and cosine) and reuses them for all num_q_heads +
+// num_k_heads heads of that row -- cos/sin are never re-read or recomputed
+// per head.  The heads
 // go in batches of U steps, software-pipelined: a batch's loads are issued
 // before the previous batch is computed, and the first batch's before the
 // row's angles, so a warp always has loads in flight (measured on batched
@@ -31,13 +32,17 @@ constexpr int kQkWarps = 4;
 // that fills the batches better (few heads per row).
 
 // angle mod 2*pi in fp64, then single precision: keeps the angle exact to
-// ~1e-7 rad for any position, and lets sincosf take its short path.
+// ~1e-7 rad for any position.  On the reduced angle, in [-pi, pi], the
+// hardware sine and cosine (__sincosf, absolute error ~1e-6 there) replace
+// the full-range sincosf: with 24 q + 4 k heads of 128 per row the per-row
+// setup is a large share of the work (long video 143.8 -> 141.3 us), and the
+// outputs move by at most one bf16 unit in ~1e-4 of the elements.
 __device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
 {
     constexpr double kTwoPi = 6.283185307179586476925286766559;
     constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
     const double red = angle - kTwoPi * rint(angle * kInvTwoPi);
-    sincosf((float)red, &s, &c);
+    __sincosf((float)red, &s, &c);
 }
 
 // Rotary layouts (template MODE).  In both rotating layouts a lane owns the
@@ -311,18 +316,22 @@ cudaError_t launch_du(const QkParams& p, int mode, unsigned grid, cudaStream_t s
     }
 }
 
-// Batch depth: 4 steps, unless 2 fills the head batches better -- a batch of
-// 4 steps spans 4 * 32 / (D / 8) heads, and a row with, say, 8 q and 8 k heads
-// of 64 would leave half of each batch's lanes without a head.
+// Batch depth: 4 steps, unless 4-step batches would leave more than a quarter
+// of their head slots empty and 2 fills them better -- a batch of 4 steps
+// spans 4 * 32 / (D / 8) heads, and a row with, say, 8 q and 8 k heads of 64
+// would leave half of each batch's lanes without a head (2 steps: 888 -> 639
+// us there), while 24 q + 4 k heads of 128 fill 7/8 of 4-step batches and run
+// faster with them (141.3 against 144.2 us on the long video).
 template <int D>
 cudaError_t launch_d(const QkParams& p, int mode, unsigned grid, cudaStream_t stream)
 {
-    auto batches = [&](int heads_per_batch) {
-        return (p.num_q_heads + heads_per_batch - 1) / heads_per_batch +
-               (p.num_k_heads + heads_per_batch - 1) / heads_per_batch;
+    auto slots = [&](int heads_per_batch) {
+        return ((p.num_q_heads + heads_per_batch - 1) / heads_per_batch +
+                (p.num_k_heads + heads_per_batch - 1) / heads_per_batch) * heads_per_batch;
     };
     constexpr int kHpw = kWarp / (D / 8);
-    const bool shallow = batches(2 * kHpw) * (2 * kHpw) < batches(4 * kHpw) * (4 * kHpw);
+    const int heads = p.num_q_heads + p.num_k_heads;
+    const bool shallow = 4 * heads < 3 * slots(4 * kHpw) && slots(2 * kHpw) < slots(4 * kHpw);
     return shallow ? launch_du<D, 2>(p, mode, grid, stream) : launch_du<D, 4>(p, mode, grid, stream);
 }
 
