@@ -1,10 +1,9 @@
 // api.cu -- the C ABI declared in include/dit_token.h: host-side argument
-// checks, the per-pair rotary frequency tables, and the launches.  Nothing
-// here allocates or synchronizes; the only state is thread-local: the last
-// CUDA error and the last rotary frequency table.
+// checks, the rotary frequency bases, and the launches.  Nothing here
+// allocates or synchronizes; the only state is thread-local: the last CUDA
+// error.
 #include <cmath>
 #include <cstdint>
-#include <cstring>
 
 #include <cuda_runtime.h>
 
@@ -19,62 +18,22 @@ namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
 
-// The rotary frequency tables of the last Q/K call on this thread, keyed by
-// what they depend on: a stream of calls with the same configuration (every
-// layer of every diffusion forward) computes them once instead of 2 * D/2
-// pow() calls per launch.  Thread-local, so concurrent callers never share
-// it; a plain value, so nothing is allocated.
-struct RopeTables {
-    bool valid = false;
-    float theta = 0.f;
-    int32_t head_dim = 0, sec_t = 0, sec_h = 0, sec_w = 0;
-    bool grid = false;
-    double inv_freq_1d[dit::kMaxPairs];
-    double inv_freq_3d[dit::kMaxPairs];
-    int8_t axis[dit::kMaxPairs];
-};
-thread_local RopeTables g_rope_tables;
-
-// Fills the per-pair tables of p: theta^(-2j/D) for 1D rows; on 3D rows pair
-// j belongs to the t, h or w section and uses theta^(-2j'/d_s), j' its index
-// inside that section of width d_s.  Computed in fp64 on the host.
-void rope_tables(dit::QkParams& p, float rope_theta, int32_t head_dim, int32_t sec_t, int32_t sec_h,
-                 int32_t sec_w, bool grid)
+// The rotary frequency bases of p, in fp64: theta^(-2/D) for 1D rows (pair j
+// turns at its j-th power, theta^(-2j/D)); on 3D rows pair j lies in the t, h
+// or w section of d_s elements (d_s / 2 pairs) and turns at
+// theta^(-2j'/d_s), the j'-th power of theta^(-2/d_s), j' its index inside
+// the section.  The kernel forms each pair's frequency from these.
+void rope_bases(dit::QkParams& p, float rope_theta, int32_t head_dim, int32_t sec_t, int32_t sec_h, int32_t sec_w,
+                bool grid)
 {
-    RopeTables& t = g_rope_tables;
-    if (!(t.valid && t.theta == rope_theta && t.head_dim == head_dim && t.sec_t == sec_t && t.sec_h == sec_h &&
-          t.sec_w == sec_w && t.grid == grid)) {
-        const double theta = (double)rope_theta;
-        const int pairs = head_dim / 2;
-        const int sec[3] = {sec_t, sec_h, sec_w};
-        for (int j = 0; j < dit::kMaxPairs; ++j) {
-            t.inv_freq_1d[j] = t.inv_freq_3d[j] = 0.0;
-            t.axis[j] = 0;
-        }
-        for (int j = 0; j < pairs; ++j) {
-            t.inv_freq_1d[j] = std::pow(theta, -2.0 * j / head_dim);
-            int first = 0, axis = 2;
-            for (int s = 0; s < 3; ++s) {
-                if (j < first + sec[s] / 2) {
-                    axis = s;
-                    break;
-                }
-                first += sec[s] / 2;
-            }
-            t.axis[j] = (int8_t)axis;
-            t.inv_freq_3d[j] = grid ? std::pow(theta, -2.0 * (j - first) / sec[axis]) : 0.0;
-        }
-        t.theta = rope_theta;
-        t.head_dim = head_dim;
-        t.sec_t = sec_t;
-        t.sec_h = sec_h;
-        t.sec_w = sec_w;
-        t.grid = grid;
-        t.valid = true;
+    const double theta = (double)rope_theta;
+    const int32_t sec[3] = {sec_t, sec_h, sec_w};
+    p.base_1d = std::pow(theta, -2.0 / head_dim);
+    for (int s = 0; s < 3; ++s) {
+        const bool used = grid && sec[s] > 0;
+        p.base_3d[s] = used ? std::pow(theta, -2.0 / sec[s]) : 0.0;
+        p.sec_pairs[s] = grid ? sec[s] / 2 : 0;
     }
-    std::memcpy(p.inv_freq_1d, t.inv_freq_1d, sizeof(p.inv_freq_1d));
-    std::memcpy(p.inv_freq_3d, t.inv_freq_3d, sizeof(p.inv_freq_3d));
-    std::memcpy(p.axis, t.axis, sizeof(p.axis));
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -201,7 +160,7 @@ dit_status dit_qk_rmsnorm_rope_shard(void* q, int64_t q_row_stride, void* k, int
     p.num_q_heads = num_q_heads;
     p.num_k_heads = num_k_heads;
     p.eps = eps;
-    rope_tables(p, rope_theta, head_dim, sec_t, sec_h, sec_w, p.rope_grid != nullptr);
+    rope_bases(p, rope_theta, head_dim, sec_t, sec_h, sec_w, p.rope_grid != nullptr);
     return from_cuda(dit::launch_qk_rmsnorm_rope(p, head_dim, rope_mode, static_cast<cudaStream_t>(stream)));
 }
 

@@ -51,7 +51,6 @@ struct Packing {
     int32_t num_rows_padded;
 };
 
-constexpr int kMaxPairs = 128;  // head_dim <= 256
 
 // Rotary layouts of dit_qk_rmsnorm_rope_ex (the DIT_ROPE_* values of the ABI).
 constexpr int kRopeInterleaved = 0;
@@ -71,12 +70,13 @@ struct QkParams {
     int32_t num_q_heads;
     int32_t num_k_heads;
     float eps;
-    // Per-pair rotary frequencies, computed once on the host in fp64:
-    // inv_freq_1d[j] = theta^(-2j/D); inv_freq_3d[j] = theta^(-2j'/d_s) for the
-    // section s = axis[j] that pair j falls in, j' its index in that section.
-    double inv_freq_1d[kMaxPairs];
-    double inv_freq_3d[kMaxPairs];
-    int8_t axis[kMaxPairs];
+    // Rotary frequency bases, fp64 from the host: pair j of a 1D row turns
+    // at base_1d^j = theta^(-2j/D); on a 3D row pair j lies in section s (the
+    // first sec_pairs[0] pairs t, the next sec_pairs[1] h, the rest w) and
+    // turns at base_3d[s]^j' = theta^(-2j'/d_s), j' its index in the section.
+    double base_1d;
+    double base_3d[3];
+    int32_t sec_pairs[3];
 };
 
 struct AdalnParams {

@@ -45,6 +45,54 @@ __device__ __forceinline__ void pair_cos_sin(double angle, float& c, float& s)
     __sincosf((float)red, &s, &c);
 }
 
+// b^k for 0 <= k < 128 (a pair index) by repeated squaring: the fp64 product
+// stays within ~1e-14 (relative) of theta^(-2j/d), far below what the fp32
+// reduced angle can resolve.
+__device__ __forceinline__ double pow_index(double b, int k)
+{
+    double r = 1.0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) {
+        if ((k >> i) & 1)
+            r *= b;
+        b *= b;
+    }
+    return r;
+}
+
+// Frequencies of the lane's NP pairs j = 4 li .. 4 li + NP - 1 and, on a 3D
+// row, their sections: 1D base_1d^j; 3D the section's base to the pair's
+// index inside the section.  The bases are read with warp-uniform indices
+// only: a parameter read whose address differs across the lanes of a warp is
+// served one address at a time (with 24 q + 4 k heads per row, reading
+// per-pair tables that way cost 4 % of the kernel on the long video and 16 %
+// on one rank's slice of it).
+template <int NP>
+__device__ __forceinline__ void pair_frequencies(const QkParams& p, int li, bool is3d, double (&f)[NP],
+                                                 int (&ax)[NP])
+{
+    const int j0 = 4 * li;
+    if (!is3d) {
+        f[0] = pow_index(p.base_1d, j0);
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            if (e > 0)
+                f[e] = f[e - 1] * p.base_1d;
+            ax[e] = 0;
+        }
+        return;
+    }
+    const int n0 = p.sec_pairs[0], n01 = n0 + p.sec_pairs[1];
+#pragma unroll
+    for (int e = 0; e < NP; ++e)
+        ax[e] = j0 + e < n0 ? 0 : (j0 + e < n01 ? 1 : 2);
+    auto base = [&](int sct) { return sct == 0 ? p.base_3d[0] : (sct == 1 ? p.base_3d[1] : p.base_3d[2]); };
+    f[0] = pow_index(base(ax[0]), j0 - (ax[0] == 0 ? 0 : (ax[0] == 1 ? n0 : n01)));
+#pragma unroll
+    for (int e = 1; e < NP; ++e)  // a pair that opens a new section is its index 0
+        f[e] = ax[e] == ax[e - 1] ? f[e - 1] * base(ax[e]) : 1.0;
+}
+
 // Rotary layouts (template MODE).  In both rotating layouts a lane owns the
 // four pairs j = 4*li .. 4*li+3 of its head:
 //   interleaved  pair j = elements (2j, 2j+1): the lane's 16-byte vector
@@ -178,7 +226,7 @@ __device__ __forceinline__ void rms_rotate_batch(uint16_t* row, int H, int h0, i
 
 template <int D, int MODE, int U>
 __global__ void __launch_bounds__(kQkWarps * kWarp)
-qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: the tables are indexed per lane
+qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place, never copied
 {
     constexpr int LPH = D / 8;          // lanes per head
     constexpr int NP = MODE == kRopeNone ? 1 : 4;  // pairs per lane
@@ -249,13 +297,13 @@ qk_rmsnorm_rope_kernel(const __grid_constant__ QkParams p)  // read in place: th
                 pos1 = g - thw;
             }
         }
+        double f[NP];
+        int ax[NP];
+        pair_frequencies<NP>(p, li, is3d, f, ax);
 #pragma unroll
         for (int e = 0; e < NP; ++e) {
-            const int j = 4 * li + e;
-            const int ax = p.axis[j];
-            const long long pj = is3d ? (ax == 0 ? pt : (ax == 1 ? ph : pw)) : pos1;
-            const double ang = (double)pj * (is3d ? p.inv_freq_3d[j] : p.inv_freq_1d[j]);
-            pair_cos_sin(ang, cs[e], sn[e]);
+            const long long pj = is3d ? (ax[e] == 0 ? pt : (ax[e] == 1 ? ph : pw)) : pos1;
+            pair_cos_sin((double)pj * f[e], cs[e], sn[e]);
         }
     }
     // the weights of the lane's 8 elements, in register order

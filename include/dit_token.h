@@ -42,9 +42,7 @@
  * Stream      `stream` is a cudaStream_t (NULL = the legacy default stream).
  *             Calls only enqueue work: they never synchronize or allocate,
  *             and are safe to call from several host threads.  The only
- *             state is per host thread: the last CUDA error and a copy of
- *             the last rotary frequency table (reused while theta, head_dim
- *             and the sections stay the same).
+ *             state is per host thread: the last CUDA error.
  * Launches    every kernel is launched with programmatic stream
  *             serialization and waits for the previous kernel on the stream
  *             to complete before its first memory access, so back-to-back
