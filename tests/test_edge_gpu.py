@@ -90,6 +90,21 @@ def test_rope_modes_and_head_dims(mode, head_dim, sections):
     P.assert_untouched(k, inp["k"], keep, "k")
 
 
+@pytest.mark.parametrize("sections", [(64, 0, 64), (0, 64, 64), (64, 64, 0), (2, 124, 2)])
+@pytest.mark.parametrize("mode", ["interleaved", "half"])
+def test_rope_sections_with_empty_or_tiny_sections(sections, mode):
+    """Each pair's frequency is formed on the device from its section's base:
+    sections of size 0 (so a lane's pairs jump from the t to the w section) or
+    of one pair agree with the oracle."""
+    w = ragged(head_dim=128, sections=sections, hq=3, hk=2, hidden=264, inner=264, seed=sum(sections[:2]) + 7)
+    rows = w.valid_rows()
+    inp = W.qk_inputs(w)
+    q, k = P.gpu_qk(w, inp, rope_mode=mode)
+    qo, ko = P.oracle_qk(w, inp, rows, rope_mode=mode)
+    P.assert_close(P.gather_rows(q, rows), qo[rows], f"q {mode} {sections}")
+    P.assert_close(P.gather_rows(k, rows), ko[rows], f"k {mode} {sections}")
+
+
 def test_half_split_video_full_size_sampled():
     w = W.workload("video")
     rows = W.sample_rows(w, per_seq=64)
