@@ -816,11 +816,13 @@ def assemble(args, world: int, w: W.Workload, whole: W.Workload, tokens: int, sc
 def run_dit(args):
     import torch.distributed as dist
     world, rank, local = dist_env()
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        # the rank's device first, and the group bound to it (its communicator
+        # then lives on this GPU, whatever device the first collective sees)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
     from dit_token_b200 import build
     if rank == 0 or world == 1:
         build.build()
