@@ -11,12 +11,12 @@
 // only its own 4 pairs: it computes them once per row (angle reduced in fp64,
 // then the hardware sine and cosine) and reuses them for all num_q_heads +
 // num_k_heads heads of that row -- cos/sin are never re-read or recomputed
-// per head.  The heads
-// go in batches of U steps, software-pipelined: a batch's loads are issued
-// before the previous batch is computed, and the first batch's before the
-// row's angles, so a warp always has loads in flight (measured on batched
-// varlen, 40x128 heads: 452 -> 429 us; with 8 K heads 300 -> 261 us).  HBM
-// traffic: q and k are each read once and written once, 4 bytes per element.
+// per head.  The heads go in batches of U steps, software-pipelined: a
+// batch's loads are issued before the previous batch is computed, and the
+// first batch's before the row's angles, so a warp always has loads in flight
+// (measured on batched varlen, 40x128 heads: 452 -> 429 us; with 8 K heads
+// 300 -> 261 us).  HBM traffic: q and k are each read once and written once,
+// 4 bytes per element.
 #include "common.cuh"
 #include "launch.h"
 
@@ -29,7 +29,8 @@ namespace {
 constexpr int kQkWarps = 4;
 
 // Steps per head batch (head vectors per lane in one batch): 4, or 2 when
-// that fills the batches better (few heads per row).
+// 4-step batches would leave over a quarter of their head slots empty (see
+// launch_d).
 
 // angle mod 2*pi in fp64, then single precision: keeps the angle exact to
 // ~1e-7 rad for any position.  On the reduced angle, in [-pi, pi], the
