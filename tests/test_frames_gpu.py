@@ -61,3 +61,17 @@ def test_empty_and_pages_request_sampled_frames():
             assert np.array_equal(got[:, t0:t0 + 1].cpu().numpy(), want), (layout, t0)
         got2 = dit.dit_frames_to_u8(x, layout=layout)
         assert torch.equal(got, got2)
+
+
+@pytest.mark.parametrize("layout", ["bthwc", "btchw"])
+def test_frames_not_32_byte_aligned(layout):
+    """Frames starting 16 bytes past a 32-byte boundary take the 16-byte loads
+    of the fast path (32-byte ones need the boundary); the bytes are the same."""
+    x_cpu = W.frames_input((1, 3, 3, 5, 32), seed=6)
+    buf = torch.zeros(x_cpu.numel() + 8, dtype=torch.float32, device="cuda")
+    x = buf[4:4 + x_cpu.numel()].view(x_cpu.shape)
+    x.copy_(x_cpu.cuda())
+    assert x.data_ptr() % 32 == 16 and x.is_contiguous()
+    got = dit.dit_frames_to_u8(x, layout=layout).cpu().numpy()
+    want = oracle.frames_to_u8(x_cpu.numpy(), layout=0 if layout == "bthwc" else 1)
+    assert np.array_equal(got, want)
