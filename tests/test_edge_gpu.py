@@ -105,6 +105,22 @@ def test_rope_sections_with_empty_or_tiny_sections(sections, mode):
     P.assert_close(P.gather_rows(k, rows), ko[rows], f"k {mode} {sections}")
 
 
+def test_rope_grid_beyond_32_bit_planes():
+    """A grid whose H x W plane passes 2^32 (1 x 70000 x 70000): the row's 3D
+    position takes the 64-bit divisions instead of the 32-bit ones, and rows
+    past W wrap to the next h; against the oracle, in both rotating layouts."""
+    lengths, padded = (300, 77000), (304, 77056)
+    w = W.custom("wide", lengths, padded, hidden=264, num_q_heads=2, num_k_heads=1, head_dim=128, inner=264,
+                 grids=((2, 3, 5), (1, 70000, 70000)), sections=(44, 42, 42), seed=12)
+    rows = W.sample_rows(w, per_seq=256)
+    for mode in ("interleaved", "half"):
+        inp = W.qk_inputs(w)
+        q, k = P.gpu_qk(w, inp, rope_mode=mode)
+        qo, ko = P.oracle_qk(w, inp, rows, rope_mode=mode)
+        P.assert_close(P.gather_rows(q, rows), qo[rows], f"q {mode}")
+        P.assert_close(P.gather_rows(k, rows), ko[rows], f"k {mode}")
+
+
 def test_half_split_video_full_size_sampled():
     w = W.workload("video")
     rows = W.sample_rows(w, per_seq=64)
