@@ -8,10 +8,11 @@
 // team of 2-8 warps for wide rows, in short-lived CTAs, so the hardware keeps
 // every SM filled with new rows as old ones finish.  A lane holds VPT vectors
 // of 4, 8 or 16 elements (8-, 16- or 32-byte accesses).  Statistics in one
-// pass: per-lane sums of x - k and (x - k)^2 about one value k of the warp
-// (lane 0's first element), added over the warp by shuffles and turned into
-// (count, mean, M2) moments, which a team merges through shared memory
-// behind one barrier.  Output pass: per element (x * rstd - mean * rstd) *
+// pass: per-lane sums of x and x^2, added over the warp by shuffles and
+// turned into (count, mean, M2) moments, which a team merges through shared
+// memory behind one barrier; a row whose mean lies more than 4 deviations
+// from 0 (where those sums lose digits) is summed again about its mean.
+// Output pass: per element (x * rstd - mean * rstd) *
 // (1 + scale) + shift in packed fp32 pairs, the per-sequence vectors read
 // through the read-only path (they stay in L1/L2: every row of a sequence
 // reads the same 2 * hidden values), 16 or 32 bytes per lane at a time.  HBM

@@ -312,9 +312,9 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8])
 }
 
 // ----------------------------------------------- row mean / variance
-// LayerNorm statistics in one pass, robust to large means and outliers: the
-// lanes of a warp accumulate s = sum(x - k) and q = sum((x - k)^2) about one
-// shift k common to the warp (a value of the row: lane 0's first element), the
+// LayerNorm statistics: the lanes of a warp accumulate s = sum(x - k) and
+// q = sum((x - k)^2) about one shift k common to the warp (first k = 0; again
+// about the row's mean where that pass lost digits, see row_moments), the
 // sums are added over the warp, and become (count, mean, M2 = sum of squared
 // deviations).  Warps that share a row merge their moments pairwise (Chan,
 // Golub and LeVeque's update):
@@ -348,10 +348,10 @@ __device__ __forceinline__ Moments moments_from_sums(float n, float k, float s, 
 // are added over the 32 lanes by an xor butterfly (both lanes of a pair add
 // the same two operands, so every lane ends with the same totals).
 // M2 = q - s^2 / n (and the mean, k + s / n) cancel when k lies far from the
-// mean -- a massive activation in the channel k is taken from: `far` reports
-// a shift more than 4 standard deviations away (s^2 / n > 16 M2), where up to
-// 4 of fp32's 24 bits are lost; the caller then sums the row again about the
-// mean just found (within a small fraction of a deviation of the true one).
+// mean: `far` reports a shift more than 4 standard deviations away
+// (s^2 / n > 16 M2), where up to 4 of fp32's 24 bits are lost; the caller
+// then sums the row again about the mean just found (within a small fraction
+// of a deviation of the true one).
 __device__ __forceinline__ Moments warp_moments(float n, float k, f32x2 s2, f32x2 q2, bool& far)
 {
     f32x2 sq = f2_make(s2.x + s2.y, q2.x + q2.y);
@@ -377,9 +377,9 @@ __device__ __forceinline__ int warp_vector_count(int warp_vec0, int nvec)
 
 // Statistics of the warp's share of a row: the VPT vectors of NW words each
 // lane holds (vectors at or past nvec are empty), about the shift k (common
-// to the warp).  Vector i of the lane is vector i * STRIDE + lane_vec0 of the
-// row.
-template <int VPT, int NW, int STRIDE>
+// to the warp; SHIFT false: k = 0, the values summed as they are).  Vector i
+// of the lane is vector i * STRIDE + lane_vec0 of the row.
+template <int VPT, int NW, int STRIDE, bool SHIFT>
 __device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW], int lane_vec0, int nvec,
                                                     float k, bool& far)
 {
@@ -391,20 +391,23 @@ __device__ __forceinline__ Moments lane_row_moments(const uint32_t (&xv)[VPT][NW
         if (i * STRIDE + lane_vec0 < nvec) {
 #pragma unroll
             for (int e = 0; e < NW; ++e) {
-                const f32x2 d = f2_sub(f2_from_bf16x2(xv[i][e]), kk);
+                const f32x2 d = SHIFT ? f2_sub(f2_from_bf16x2(xv[i][e]), kk) : f2_from_bf16x2(xv[i][e]);
                 s2 = f2_add(s2, d);
                 q2 = f2_fma(d, d, q2);
             }
         }
     }
     const int nv = warp_vector_count<VPT, STRIDE>(lane_vec0 - lane, nvec);
-    return warp_moments((float)(2 * NW * nv), k, s2, q2, far);
+    return warp_moments((float)(2 * NW * nv), SHIFT ? k : 0.f, s2, q2, far);
 }
 
-// The row's moments: sums about lane 0's first element of each warp, merged
-// across a team of TEAM warps (TEAM > 1: through shared memory, behind a
-// barrier); summed again about the mean found when a warp's shift lay far
-// from it.  red, red2 and far_w: TEAM entries of shared memory.
+// The row's moments: sums of the values and their squares as they are (about
+// 0), merged across a team of TEAM warps (TEAM > 1: through shared memory,
+// behind a barrier); summed again about the mean found when a warp's mean lay
+// more than 4 deviations from 0, where the first sums lose digits.  A row
+// whose mean is small against its spread -- the usual case, massive
+// activations in a few channels included -- takes one pass.  red, red2 and
+// far_w: TEAM entries of shared memory.
 template <int VPT, int NW, int TEAM>
 __device__ __forceinline__ Moments row_moments(const uint32_t (&xv)[VPT][NW], int nvec, Moments* red,
                                                Moments* red2, int* far_w)
@@ -416,8 +419,7 @@ __device__ __forceinline__ Moments row_moments(const uint32_t (&xv)[VPT][NW], in
     // team per row (one row per CTA)
     const int tt = TEAM == 1 ? lane : (int)threadIdx.x;
     bool far;
-    Moments m = lane_row_moments<VPT, NW, STRIDE>(xv, tt, nvec, __shfl_sync(0xffffffffu, bf16_lo(xv[0][0]), 0),
-                                                  far);
+    Moments m = lane_row_moments<VPT, NW, STRIDE, false>(xv, tt, nvec, 0.f, far);
     if constexpr (TEAM > 1) {
         if (lane == 0) {
             red[warp] = m;
@@ -434,7 +436,7 @@ __device__ __forceinline__ Moments row_moments(const uint32_t (&xv)[VPT][NW], in
     }
     if (far) {  // uniform over the warp (TEAM 1) or the CTA
         bool unused;
-        m = lane_row_moments<VPT, NW, STRIDE>(xv, tt, nvec, m.mean, unused);
+        m = lane_row_moments<VPT, NW, STRIDE, true>(xv, tt, nvec, m.mean, unused);
         if constexpr (TEAM > 1) {
             if (lane == 0)
                 red2[warp] = m;
