@@ -1,4 +1,4 @@
-"""Row sharding of a packed batch across ranks (host logic, numpy only).
+"""Row and head sharding of a packed batch across ranks (host logic, numpy only).
 
 The operators are row-local, so a packed batch splits across ranks with no
 exchange: rank r takes a contiguous range of the valid tokens, balanced by
@@ -98,3 +98,31 @@ def shard_packing(cu_seqlens, cu_seqlens_padded, rope_grid, rank: int, world: in
     return Shard(rank, world, np.asarray(seq, dtype=np.int32), np.asarray(off, dtype=np.int32), cu, cu_p,
                  None if grid is None else grid[np.asarray(seq, dtype=np.int64)].astype(np.int32),
                  np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64))
+
+
+def head_range(num_q_heads: int, num_k_heads: int, rank: int, world: int) -> tuple:
+    """(q_first, q_count, k_first, k_count): the heads rank `rank` of `world`
+    holds when Q/K are split by heads instead of rows (the layout after a
+    sequence-to-head all-to-all).  Every rank keeps all rows, so positions
+    need no offsets; the per-head normalisation and rotation are independent
+    of the other heads, and a rank's call on its heads (a column slice of the
+    whole buffer, or its own contiguous buffer) equals those columns of the
+    whole call.  q heads split evenly; k heads split evenly when there are at
+    least as many as ranks, else each is replicated on world / num_k_heads
+    ranks -- either way the rank holds exactly the k heads its q heads attend
+    with under grouped-query attention (q head h uses k head
+    h // (num_q_heads / num_k_heads))."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of world {world}")
+    if num_q_heads < 1 or num_k_heads < 1 or num_q_heads % num_k_heads:
+        raise ValueError("num_q_heads must be a positive multiple of num_k_heads")
+    if num_q_heads % world:
+        raise ValueError(f"{num_q_heads} q heads do not split over {world} ranks")
+    if num_k_heads >= world:
+        if num_k_heads % world:
+            raise ValueError(f"{num_k_heads} k heads do not split over {world} ranks")
+        kc = num_k_heads // world
+        return rank * (num_q_heads // world), num_q_heads // world, rank * kc, kc
+    if world % num_k_heads:
+        raise ValueError(f"{num_k_heads} k heads do not replicate evenly over {world} ranks")
+    return rank * (num_q_heads // world), num_q_heads // world, rank * num_k_heads // world, 1

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import oracle
-from dit_token_b200.shard import shard_packing
+from dit_token_b200.shard import head_range, shard_packing
 from _util import bits, cu
 
 # sequences: 3D video (24 rows) + 9 audio rows, a 1D one, an empty one, 3D only
@@ -117,3 +117,48 @@ def test_more_ranks_than_tokens_and_empty_batches():
     assert np.array_equal(empty[2].rows, np.arange(8))
     with pytest.raises(ValueError):
         shard_packing(cs, cp, None, 3, 3)
+
+
+@pytest.mark.parametrize("Hq,Hk,world", [(8, 8, 2), (8, 2, 2), (8, 2, 4), (8, 2, 8), (24, 4, 8), (40, 8, 4), (6, 1, 3)])
+def test_head_range_covers_every_head_with_its_group(Hq, Hk, world):
+    """q heads partition over the ranks; a rank holds exactly the k heads its
+    q heads use under grouped-query attention (q head h -> k head h // (Hq/Hk))."""
+    seen = []
+    for r in range(world):
+        q0, qc, k0, kc = head_range(Hq, Hk, r, world)
+        seen += list(range(q0, q0 + qc))
+        assert set(range(k0, k0 + kc)) == {h // (Hq // Hk) for h in range(q0, q0 + qc)}
+    assert seen == list(range(Hq))
+
+
+def test_head_range_rejects_uneven_splits():
+    for args in [(8, 2, 3), (8, 3, 2), (6, 2, 4), (12, 4, 8), (8, 2, 2 * 8)]:
+        with pytest.raises(ValueError):
+            head_range(*args[:2], 0, args[2])
+    with pytest.raises(ValueError):
+        head_range(8, 2, 2, 2)
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("mode", ["interleaved", "half"])
+def test_head_slices_reproduce_the_whole_call(world, mode):
+    """The normalisation and rotation of one head read no other head: each
+    rank's oracle call on its heads (every row, its own columns) equals those
+    columns of the call on all heads.  A norm taken over the whole row instead
+    of per head fails this."""
+    Hq, Hk = 4, 2
+    rng = np.random.default_rng(21)
+    rows = sum(PADDED)
+    q = bits(rng.standard_normal((rows, Hq * D)) * np.repeat(rng.uniform(0.2, 5.0, Hq), D))
+    k = bits(rng.standard_normal((rows, Hk * D)) * np.repeat(rng.uniform(0.2, 5.0, Hk), D))
+    wq, wk = bits(np.linspace(0.5, 1.5, D)), bits(np.linspace(1.5, 0.5, D))
+    cs, cp = cu(LENGTHS), cu(PADDED)
+    kw = dict(head_dim=D, rope_grid=GRID, sections=SEC, rope_mode=mode)
+    qf, kf = oracle.qk_rmsnorm_rope(q, k, wq, wk, cs, cp, num_q_heads=Hq, num_k_heads=Hk, **kw)
+    for r in range(world):
+        q0, qc, k0, kc = head_range(Hq, Hk, r, world)
+        qsl, ksl = slice(q0 * D, (q0 + qc) * D), slice(k0 * D, (k0 + kc) * D)
+        qo, ko = oracle.qk_rmsnorm_rope(np.ascontiguousarray(q[:, qsl]), np.ascontiguousarray(k[:, ksl]), wq, wk,
+                                        cs, cp, num_q_heads=qc, num_k_heads=kc, **kw)
+        assert np.array_equal(qo, qf[:, qsl]), (r, "q")
+        assert np.array_equal(ko, kf[:, ksl]), (r, "k")

@@ -9,7 +9,7 @@ import torch
 
 import dit_token_b200 as dit
 from dit_token_b200 import workloads as W
-from dit_token_b200.shard import shard_packing
+from dit_token_b200.shard import head_range, shard_packing
 import _parity as P
 import oracle
 from _util import tbits
@@ -106,3 +106,45 @@ def test_slice_qk_matches_the_oracle_slice_call():
                                 for i in range(sh.num_seqs)])
         P.assert_close(tbits(q)[valid], qo[valid], f"slice {rank} q")
         P.assert_close(tbits(k)[valid], ko[valid], f"slice {rank} k")
+
+
+def heads():
+    return W.custom("hs", (700, 45, 0, 300), (704, 48, 8, 304), hidden=256, num_q_heads=8, num_k_heads=2,
+                    head_dim=128, inner=264, grids=((4, 6, 25), (0, 0, 0), (0, 0, 0), (3, 5, 10)),
+                    sections=(32, 48, 48), seed=3)
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+@pytest.mark.parametrize("rope_mode", ["interleaved", "half"])
+@pytest.mark.parametrize("layout", ["view", "copy"])
+def test_head_slices_equal_the_whole_call(world, rope_mode, layout):
+    """Sharding by heads (the layout after a sequence-to-head all-to-all):
+    rank r holds every row but only its q heads and the k head(s) they use
+    (dit_token_b200.shard.head_range; k heads are replicated when there are
+    fewer than ranks).  Each rank's call on its heads, either in place on a
+    column view of the whole buffer (row stride of all heads) or on its own
+    contiguous buffer, equals the unsharded call's columns bit for bit, though
+    the kernel's batching of heads per CTA changes with the head count."""
+    w = heads()
+    rv = W.rows_view
+    qi = W.qk_inputs(w)
+    q0, k0 = rv(qi["q"]).cuda(), rv(qi["k"]).cuda()
+    wq, wk = qi["q_weight"].cuda(), qi["k_weight"].cuda()
+    cs, cp, grid = P.device_packing(w)
+    D, Hq, Hk = w.head_dim, w.num_q_heads, w.num_k_heads
+    kw = dict(head_dim=D, rope_grid=grid, sections=w.sections, rope_theta=w.rope_theta, eps=w.eps,
+              rope_mode=rope_mode)
+    qf, kf = q0.clone(), k0.clone()
+    dit.dit_qk_rmsnorm_rope(qf, kf, wq, wk, cs, cp, num_q_heads=Hq, num_k_heads=Hk, **kw)
+    qs = q0.clone()
+    for rank in range(world):
+        qh0, hq, kh0, hk = head_range(Hq, Hk, rank, world)
+        qcols, kcols = slice(qh0 * D, (qh0 + hq) * D), slice(kh0 * D, (kh0 + hk) * D)
+        q = qs[:, qcols] if layout == "view" else q0[:, qcols].contiguous()
+        k = k0[:, kcols].contiguous()
+        dit.dit_qk_rmsnorm_rope(q, k, wq, wk, cs, cp, num_q_heads=hq, num_k_heads=hk, **kw)
+        if layout == "copy":
+            assert torch.equal(q.view(torch.int16), qf[:, qcols].view(torch.int16)), (world, rank, "q")
+        assert torch.equal(k.view(torch.int16), kf[:, kcols].view(torch.int16)), (world, rank, "k")
+    if layout == "view":
+        assert torch.equal(qs.view(torch.int16), qf.view(torch.int16)), world
