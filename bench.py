@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N [--split]] [--steps K] [--warmup W] [--impl dit|reference]
                     [--workload batched_varlen] [--seed 0]
-                    [--table | --variants | --host-overhead]
+                    [--table | --variants | --host-overhead | --launch-cost]
 
 One step runs the whole per-token hot path once over one packed batch:
 Q/K RMSNorm + RoPE (in place), adaLN modulation, gated residual and SwiGLU,
@@ -40,7 +40,9 @@ the host cores and prints the same JSON line with "impl": "reference".
 ``--variants`` one over the operator variants (fp32 and per-stream
 modulation vectors, rotary layouts, grouped K heads, head_dim 256), both
 with a read-only pass over 512 MB before every timed launch (clean L2);
-``--host-overhead`` prints the host time per call of every entry point.
+``--host-overhead`` prints the host time per call of every entry point, and
+``--launch-cost`` the device time of one call alone and of the same call
+twice back to back at the small shapes.
 """
 from __future__ import annotations
 
@@ -1115,6 +1117,68 @@ def run_host_overhead(args):
         print(f"| {name} | {(t1 - t0) / n * 1e6:.2f} | {(t3 - t2) / n * 1e6:.2f} |", flush=True)
 
 
+def run_launch_cost(args):
+    """What one launch costs when timed alone, and what the same call adds
+    right behind another: device time between two CUDA events around the
+    call(s), after a read-only pass over 512 MB (clean L2), median of --steps.
+    Rows: nothing between the events, a one-element torch fill, the library's
+    smallest kernel, and every op of the tiny and per-rank-sized workloads.
+    "twice" runs the op on two separate buffer sets back to back, so the
+    increment is the second launch's cost in a chain, read from HBM like the
+    first.  The library loaded is the in-tree one, or DIT_TOKEN_LIB (e.g. a
+    build with --define DIT_PDL=0)."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from dit_token_b200 import build
+    build.build()
+    import dit_token_b200 as dit
+    peak, kind = measured_peak()
+    flush = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)  # 512 MB, 4x L2
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.sum()  # a read-only pass: L2 ends up holding clean lines
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(device)
+        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3  # us
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    print(f"library: {dit.LIB_PATH}")
+    print(f"| workload | call | once us | twice us | increment us | increment GB/s | % of {kind} {peak:.0f} GB/s |")
+    print("|---|---|---|---|---|---|---|")
+    one = torch.zeros(1, device=device)
+    print(f"| - | nothing | {timed(lambda: None):.2f} | - | - | - | - |")
+    print(f"| - | torch fill, 1 element | {timed(lambda: one.fill_(1.0)):.2f} | - | - | - | - |")
+    cs = torch.tensor([0, 100, 200], dtype=torch.int32, device=device)
+    grid = torch.tensor([[2, 5, 5], [1, 2, 3]], dtype=torch.int32, device=device)
+    outs = [(torch.empty(5, dtype=torch.int32, device=device), torch.empty(5, dtype=torch.int32, device=device))
+            for _ in range(2)]
+    av = [lambda o=o: dit.dit_av_stream_seqlens(cs, cs, grid, out=o) for o in outs]
+    t1, t2 = timed(av[0]), timed(lambda: (av[0](), av[1]()))
+    print(f"| - | dit_av_stream_seqlens, 2 sequences | {t1:.2f} | {t2:.2f} | {t2 - t1:.2f} | - | - |", flush=True)
+    for name in ("tiny",) + SMALL_SHAPES:
+        w = W.workload(name, args.seed)
+        host = host_inputs(w)
+        sa, sb = Step(w, host, device), Step(w, host, device)
+        ab = algorithmic_bytes(w)
+        for op in OPS:
+            t1 = timed(lambda: sa.run_op(op))
+            t2 = timed(lambda: (sa.run_op(op), sb.run_op(op)))
+            gbs = ab[op] / ((t2 - t1) * 1e-6) / 1e9
+            print(f"| {name} | {op} | {t1:.2f} | {t2:.2f} | {t2 - t1:.2f} | {gbs:.0f} | {100 * gbs / peak:.1f} |",
+                  flush=True)
+        del sa, sb, host
+        torch.cuda.empty_cache()
+    print(clock_note(sampler), flush=True)
+
+
 def run_profile_op(args):
     """One operator alone, at the workload's full shape, with only its own
     buffers on the device (adaLN on batched varlen: 2 x 718 MB): W + K
@@ -1188,6 +1252,9 @@ def main(argv=None):
                     help="print a markdown table of the operator variants instead of the JSON line")
     ap.add_argument("--host-overhead", action="store_true",
                     help="print the host time per call of every entry point (tiny workload, no sync)")
+    ap.add_argument("--launch-cost", action="store_true",
+                    help="print the device time of one call and of two back to back (tiny and per-rank "
+                         "sized workloads) instead of the JSON line")
     ap.add_argument("--profile-op", choices=OPS,
                     help="launch only this operator, W + K times on the workload with its own buffers "
                          "(for a profiler capture of one full-size launch)")
@@ -1202,6 +1269,8 @@ def main(argv=None):
         run_profile_op(args)
     elif args.host_overhead:
         run_host_overhead(args)
+    elif args.launch_cost:
+        run_launch_cost(args)
     elif args.table:
         run_table(args)
     elif args.variants:

@@ -223,3 +223,14 @@ def test_binding_rejects_cpu_tensors_before_the_library():
         dit._seq_vectors(torch.zeros(1, 8, dtype=torch.float16), 8, "gate")
     with pytest.raises(TypeError):   # mixed bf16 / fp32 vectors in one call
         dit._one_dtype((0, 1, 0), "gate, shift and scale")
+
+
+def test_switched_build_never_replaces_the_in_tree_library():
+    """A build with compile-time switches (e.g. DIT_PDL=0) must name its own
+    output file; the in-tree library is left as it is."""
+    before = os.path.getmtime(build.LIB) if os.path.exists(build.LIB) else None
+    for out in (None, build.LIB):
+        with pytest.raises(ValueError):
+            build.build(out=out, defines=["DIT_PDL=0"])
+    after = os.path.getmtime(build.LIB) if os.path.exists(build.LIB) else None
+    assert before == after
