@@ -2,7 +2,8 @@
 benchmark each rank draws its own batch of the same shapes (no data is
 exchanged), the timing is the max over ranks, and every rank takes the same
 collective steps; when ranks split one batch instead, each rank's slice
-(with its rows' whole-sequence positions) gives the unsharded result."""
+(with its rows' whole-sequence positions) gives the unsharded result, and so
+does each rank's share of the heads."""
 import os
 import socket
 
@@ -111,6 +112,53 @@ def test_two_ranks_split_one_batch_with_global_positions():
     port = _free_port()
     mp.spawn(_shard_worker, args=(2, port, out), nprocs=2, join=True)
     assert out["rows"] and out["equal"]
+
+
+def _head_worker(rank, world, port, out):
+    """Split by heads instead (the layout after a sequence-to-head
+    all-to-all): every rank holds all rows and runs the oracle on its q heads
+    and the k head they use; the columns are gathered."""
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from dit_token_b200 import workloads as W
+    from dit_token_b200.shard import head_range
+    from _util import tbits
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        D, Hq, Hk = 64, 4, 2
+        w = W.custom("hp", (700, 45, 300), (704, 48, 304), hidden=128, num_q_heads=Hq, num_k_heads=Hk,
+                     head_dim=D, inner=64, grids=((4, 6, 25), (0, 0, 0), (3, 5, 10)), sections=(24, 20, 20))
+        inp = W.qk_inputs(w)
+        q, k = tbits(W.rows_view(inp["q"])), tbits(W.rows_view(inp["k"]))
+        wq, wk = tbits(inp["q_weight"]), tbits(inp["k_weight"])
+        q0, qc, k0, kc = head_range(Hq, Hk, rank, world)
+        qo, ko = oracle.qk_rmsnorm_rope(np.ascontiguousarray(q[:, q0 * D:(q0 + qc) * D]),
+                                        np.ascontiguousarray(k[:, k0 * D:(k0 + kc) * D]), wq, wk, w.cu_seqlens,
+                                        w.cu_seqlens_padded, num_q_heads=qc, num_k_heads=kc, head_dim=D,
+                                        rope_grid=w.rope_grid, sections=w.sections)
+        parts_q = [torch.zeros(qo.shape, dtype=torch.int64) for _ in range(world)]
+        parts_k = [torch.zeros(ko.shape, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(parts_q, torch.from_numpy(qo.astype(np.int64)))
+        dist.all_gather(parts_k, torch.from_numpy(ko.astype(np.int64)))
+        if rank == 0:
+            fq, fk = oracle.qk_rmsnorm_rope(q, k, wq, wk, w.cu_seqlens, w.cu_seqlens_padded, num_q_heads=Hq,
+                                            num_k_heads=Hk, head_dim=D, rope_grid=w.rope_grid,
+                                            sections=w.sections)
+            out["q"] = bool(np.array_equal(np.concatenate([t.numpy() for t in parts_q], axis=1), fq))
+            out["k"] = bool(np.array_equal(np.concatenate([t.numpy() for t in parts_k], axis=1), fk))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_split_heads():
+    mgr = mp.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    mp.spawn(_head_worker, args=(2, port, out), nprocs=2, join=True)
+    assert out["q"] and out["k"]
 
 
 def _split_worker(rank, world, port, out):
