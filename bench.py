@@ -41,8 +41,8 @@ the host cores and prints the same JSON line with "impl": "reference".
 modulation vectors, rotary layouts, grouped K heads, head_dim 256), both
 with a read-only pass over 512 MB before every timed launch (clean L2);
 ``--host-overhead`` prints the host time per call of every entry point, and
-``--launch-cost`` the device time of one call alone and of the same call
-twice back to back at the small shapes.
+``--launch-cost`` the device time of one call alone and per call in a chain
+of calls on separate buffer sets at the small shapes.
 """
 from __future__ import annotations
 
@@ -665,6 +665,7 @@ def plan(args, rank: int, world: int):
 
 
 SMALL_SHAPES = ("single_stream", "long_video_slice")
+LAUNCH_CHAIN = 8  # buffer sets in --launch-cost's chain (per-rank shapes: 8 x 67-380 MB, beyond the 126 MB L2)
 
 
 def time_small_shapes(device, seed: int, steps: int = 100, reps: int = 30) -> dict:
@@ -1118,15 +1119,17 @@ def run_host_overhead(args):
 
 
 def run_launch_cost(args):
-    """What one launch costs when timed alone, and what the same call adds
-    right behind another: device time between two CUDA events around the
-    call(s), after a read-only pass over 512 MB (clean L2), median of --steps.
-    Rows: nothing between the events, a one-element torch fill, the library's
+    """What one launch costs when timed alone, and what the same call costs
+    inside a chain: device time between two CUDA events around the call(s),
+    after a read-only pass over 512 MB (clean L2), median of --steps.  Rows:
+    nothing between the events, a one-element torch fill, the library's
     smallest kernel, and every op of the tiny and per-rank-sized workloads.
-    "twice" runs the op on two separate buffer sets back to back, so the
-    increment is the second launch's cost in a chain, read from HBM like the
-    first.  The library loaded is the in-tree one, or DIT_TOKEN_LIB (e.g. a
-    build with --define DIT_PDL=0)."""
+    The chain runs the op on CHAIN separate buffer sets back to back (more
+    bytes than L2 holds), so each call after the first reads from HBM and
+    writes back its predecessor's dirty lines, as in a stream of ops; the
+    per-call cost in the chain is (chain - once) / (CHAIN - 1).  The library
+    loaded is the in-tree one, or DIT_TOKEN_LIB (e.g. a build with --define
+    DIT_PDL=0)."""
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     from dit_token_b200 import build
@@ -1135,46 +1138,59 @@ def run_launch_cost(args):
     peak, kind = measured_peak()
     flush = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)  # 512 MB, 4x L2
 
+    host_us = []
+
     def timed(fn):
         for _ in range(args.warmup):
             fn()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+        host_us.clear()
         for a, b in ev:
             flush.sum()  # a read-only pass: L2 ends up holding clean lines
+            # about 0.5 ms of one spinning thread: the host has queued every
+            # call of the chain before the first event, so the GPU never
+            # waits for the Python side between them
+            torch.cuda._sleep(1_000_000)
             a.record()
+            t0 = time.perf_counter()
             fn()
+            host_us.append((time.perf_counter() - t0) * 1e6)
             b.record()
         torch.cuda.synchronize(device)
         return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3  # us
 
     sampler = ClockSampler(0)
     sampler.start()
+    n = LAUNCH_CHAIN
     print(f"library: {dit.LIB_PATH}")
-    print(f"| workload | call | once us | twice us | increment us | increment GB/s | % of {kind} {peak:.0f} GB/s |")
-    print("|---|---|---|---|---|---|---|")
+    print(f"| workload | call | once us | chain of {n} us | host us to queue the chain | per call in the chain us | "
+          f"GB/s in the chain | % of {kind} {peak:.0f} GB/s |")
+    print("|---|---|---|---|---|---|---|---|")
     one = torch.zeros(1, device=device)
-    print(f"| - | nothing | {timed(lambda: None):.2f} | - | - | - | - |")
-    print(f"| - | torch fill, 1 element | {timed(lambda: one.fill_(1.0)):.2f} | - | - | - | - |")
+    print(f"| - | nothing | {timed(lambda: None):.2f} | - | - | - | - | - |")
+    print(f"| - | torch fill, 1 element | {timed(lambda: one.fill_(1.0)):.2f} | - | - | - | - | - |")
     cs = torch.tensor([0, 100, 200], dtype=torch.int32, device=device)
     grid = torch.tensor([[2, 5, 5], [1, 2, 3]], dtype=torch.int32, device=device)
     outs = [(torch.empty(5, dtype=torch.int32, device=device), torch.empty(5, dtype=torch.int32, device=device))
-            for _ in range(2)]
+            for _ in range(n)]
     av = [lambda o=o: dit.dit_av_stream_seqlens(cs, cs, grid, out=o) for o in outs]
-    t1, t2 = timed(av[0]), timed(lambda: (av[0](), av[1]()))
-    print(f"| - | dit_av_stream_seqlens, 2 sequences | {t1:.2f} | {t2:.2f} | {t2 - t1:.2f} | - | - |", flush=True)
+    t1, tn = timed(av[0]), timed(lambda: [f() for f in av])
+    print(f"| - | dit_av_stream_seqlens, 2 sequences | {t1:.2f} | {tn:.2f} | {statistics.median(host_us):.1f} | "
+          f"{(tn - t1) / (n - 1):.2f} | - | - |", flush=True)
     for name in ("tiny",) + SMALL_SHAPES:
         w = W.workload(name, args.seed)
         host = host_inputs(w)
-        sa, sb = Step(w, host, device), Step(w, host, device)
+        sets = [Step(w, host, device) for _ in range(n)]
         ab = algorithmic_bytes(w)
         for op in OPS:
-            t1 = timed(lambda: sa.run_op(op))
-            t2 = timed(lambda: (sa.run_op(op), sb.run_op(op)))
-            gbs = ab[op] / ((t2 - t1) * 1e-6) / 1e9
-            print(f"| {name} | {op} | {t1:.2f} | {t2:.2f} | {t2 - t1:.2f} | {gbs:.0f} | {100 * gbs / peak:.1f} |",
-                  flush=True)
-        del sa, sb, host
+            t1 = timed(lambda: sets[0].run_op(op))
+            tn = timed(lambda: [st.run_op(op) for st in sets])
+            per = (tn - t1) / (n - 1)
+            gbs = ab[op] / (per * 1e-6) / 1e9
+            print(f"| {name} | {op} | {t1:.2f} | {tn:.2f} | {statistics.median(host_us):.1f} | {per:.2f} | "
+                  f"{gbs:.0f} | {100 * gbs / peak:.1f} |", flush=True)
+        del sets, host
         torch.cuda.empty_cache()
     print(clock_note(sampler), flush=True)
 
@@ -1253,8 +1269,8 @@ def main(argv=None):
     ap.add_argument("--host-overhead", action="store_true",
                     help="print the host time per call of every entry point (tiny workload, no sync)")
     ap.add_argument("--launch-cost", action="store_true",
-                    help="print the device time of one call and of two back to back (tiny and per-rank "
-                         "sized workloads) instead of the JSON line")
+                    help="print the device time of one call alone and per call in a chain (tiny and "
+                         "per-rank sized workloads) instead of the JSON line")
     ap.add_argument("--profile-op", choices=OPS,
                     help="launch only this operator, W + K times on the workload with its own buffers "
                          "(for a profiler capture of one full-size launch)")

@@ -241,6 +241,19 @@ AdalnShape adaln_shape(const AdalnParams& p)
         sh.wide_vectors = false;
         sh.team = fit(4);
     }
+    // A warp holding 6-8 vectors of 32 bytes per lane (rows of 3072-4096
+    // elements) runs at 82-98 registers, so 16-20 warps fit on an SM; a team
+    // of 2 holds 3-4 each at 54-63 registers, 32-36 warps.  Measured per call
+    // in a chain of launches (clean L2 before the chain, 1965 MHz), the team
+    // is 8-13 % faster at 4-8 K rows, 2-5 % at 16-32 K and about 1 % at 61,888
+    // (3072) or 65,536 (4096) rows, and 1.2 % slower at 131,072 rows of 3072.
+    // At 4-5 vectors (2048-2560) the team was behind at every row count but
+    // one (8 K rows of 2048: 2 % ahead), so those keep one warp per row.
+    if (sh.team == 1 && sh.row_words == 8 && p.pk.num_rows_padded <= 65536) {
+        const int nvec = p.hidden / 16;
+        if ((nvec + kWarp - 1) / kWarp >= 6)
+            sh.team = 2;
+    }
     return sh;
 }
 
